@@ -1,0 +1,472 @@
+"""Throughput of the paged-attention hot path on B200.
+
+One step = one decode iteration of the Llama-3-8B-shaped GQA batch (256
+sequences, 32 q / 8 kv heads, head_dim 128, bf16, 16-token blocks, lengths
+uniform in [128, 4096], shuffled physical blocks): slot mapping of the new
+token of every sequence, reshape_and_cache of its K/V, split-KV paged decode
+and the log-sum-exp reduce — all through libpa.so's C ABI.
+
+Printed (rank 0, one JSON line): the decode KV bandwidth over the whole step
+(GB/s of algorithmic K/V bytes), decode tokens/s, the roofline of pa_decode,
+the prefill-chunk TFLOP/s of the 8 x 512-token chunk workload, an end-to-end
+figure through the C ABI with host buffers, clocks seen during the timed
+region, and the CPU oracle as a baseline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+For N > 1 launch with torch.distributed.run; every rank decodes its own batch
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "paged decode KV GB/s (% of HBM peak) and decode tokens/s; prefill-chunk TFLOP/s"
+WORKLOAD = ("llama3_8b_gqa_decode: 256 seqs, 32 q / 8 kv heads, head_dim 128, bf16, "
+            "block_size 16, lengths U[128,4096], shuffled block tables, +1 appended token/seq")
+PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_llama3_8b_gqa_decode.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_397_b200", "csrc", f)
+                  for f in ("decode.cuh", "ptx.cuh")]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kv_bytes_per_launch: float):
+    """DRAM bytes per decode launch from the committed ncu summary, scaled to
+    this launch by K/V bytes, or None if the kernel changed since the capture."""
+    if not os.path.exists(PROFILE):
+        return None
+    text = open(PROFILE).read()
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_ratio = re.search(r"dram_bytes_per_algorithmic_byte:\s*([0-9.]+)", text)
+    if not m_hash or not m_ratio or m_hash.group(1) != kernel_hash():
+        return None
+    return float(m_ratio.group(1)) * kv_bytes_per_launch
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class DecodeStep:
+    """Device-resident inputs of one decode step and the C-ABI calls it makes."""
+
+    def __init__(self, w, dev):
+        import paged_kv_cache_397_b200 as pa
+        self.pa = pa
+        self.w = w
+        self.dev = dev
+        self.kc = w.key_cache.to(dev)
+        self.vc = w.value_cache.to(dev)
+        self.bt = w.block_tables.to(dev)
+        self.ctx = w.context_lens.to(dev)
+        self.lens = (w.context_lens + 1).to(dev)
+        self.q = w.query.to(dev)
+        self.nk = w.new_key.to(dev)
+        self.nv = w.new_value.to(dev)
+        self.slots = torch.empty(w.num_seqs, dtype=torch.int64, device=dev)
+        self.out = torch.empty_like(self.q)
+        self.max_len = int(w.context_lens.max()) + 1
+        need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads,
+                                           w.head_dim, w.block_size, self.max_len)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.num_parts = math.ceil(self.max_len / pa.pa_decode_partition_tokens(
+            w.num_seqs, w.num_kv_heads, w.block_size, self.max_len))
+        self.launches_per_step = 3 + (1 if self.num_parts > 1 else 0)
+        total = int(self.lens.sum())
+        self.kv_bytes = 2 * w.num_kv_heads * w.head_dim * 2 * total  # K and V, bf16
+        # host-side copies for the end-to-end leg (pinned)
+        self.h_q = w.query.pin_memory()
+        self.h_nk = w.new_key.pin_memory()
+        self.h_nv = w.new_value.pin_memory()
+        self.h_bt = w.block_tables.pin_memory()
+        self.h_ctx = w.context_lens.pin_memory()
+        self.h_lens = (w.context_lens + 1).pin_memory()
+        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in
+                             (self.h_q, self.h_nk, self.h_nv, self.h_bt, self.h_ctx, self.h_lens))
+        self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
+
+    def append(self):
+        pa, w = self.pa, self.w
+        pa.pa_slot_mapping(self.slots, self.bt, self.ctx, w.block_size)
+        pa.pa_reshape_and_cache(self.nk, self.nv, self.kc, self.vc, self.slots)
+
+    def decode(self):
+        self.pa.pa_decode(self.out, self.q, self.kc, self.vc, self.bt, self.lens, self.max_len,
+                          self.w.scale, workspace=self.ws)
+
+    def step(self):
+        self.append()
+        self.decode()
+
+    def step_e2e(self):
+        for h, d in ((self.h_q, self.q), (self.h_nk, self.nk), (self.h_nv, self.nv),
+                     (self.h_bt, self.bt), (self.h_ctx, self.ctx), (self.h_lens, self.lens)):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.out, non_blocking=True)
+
+
+def time_steps(fn, steps, stream):
+    """CUDA-event time of `steps` calls of fn on `stream` (ms total)."""
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b)
+
+
+def prefill_measure(dev, steps, warmup, block_size):
+    import paged_kv_cache_397_b200 as pa
+    p = synth.chunked_prefill(block_size=block_size)
+    kc, vc = p.key_cache.to(dev), p.value_cache.to(dev)
+    bt, cl, cu = p.block_tables.to(dev), p.ctx_lens.to(dev), p.cu_q_lens.to(dev)
+    q = p.query.to(dev)
+    nk, nv = p.new_key.to(dev), p.new_value.to(dev)
+    slots = torch.empty(p.total_q, dtype=torch.int64, device=dev)
+    pa.pa_slot_mapping(slots, bt, cl, p.block_size, cu_q_lens=cu)
+    pa.pa_reshape_and_cache(nk, nv, kc, vc, slots)
+    out = torch.empty_like(q)
+    qmax, cmax = int(torch.diff(p.cu_q_lens).max()), int(p.ctx_lens.max())
+    fn = lambda: pa.pa_prefill_chunk(out, q, kc, vc, bt, cu, cl, qmax, cmax, p.scale)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ms = time_steps(fn, steps, torch.cuda.current_stream()) / steps
+    flops = 0
+    for c, n in zip(p.ctx_lens.tolist(), torch.diff(p.cu_q_lens).tolist()):
+        flops += 4 * p.head_dim * p.num_q_heads * (n * c + n * (n + 1) // 2)
+    return {"workload": p.name, "block_size": block_size, "ms": ms,
+            "tflops": flops / ms / 1e9, "causal_flop": flops}
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The oracle, as it stands, on a seeded sample of the batch's sequences."""
+    import threadpoolctl
+
+    import oracle
+    lens = (w.context_lens + 1).tolist()
+    rng = np.random.default_rng(0)
+    seqs = sorted(rng.choice(w.num_seqs, size=min(64, w.num_seqs), replace=False).tolist())
+    # the appended token: written with the oracle's own slot arithmetic
+    kcv = w.key_cache.view(torch.int16).numpy()
+    vcv = w.value_cache.view(torch.int16).numpy()
+    slots = oracle.logical_positions_to_slots(w.block_tables.numpy(), np.arange(w.num_seqs),
+                                              w.context_lens.numpy(), w.block_size)
+    used = sorted({int(b) for s in seqs for b in w.block_tables[s, :-(-lens[s] // 16)]})
+    remap = {b: i for i, b in enumerate(used)}
+    idx = torch.tensor(used)
+    kc = w.key_cache.index_select(0, idx).double().numpy()
+    vc = w.value_cache.index_select(0, idx).double().numpy()
+    bt = np.full((len(seqs), w.block_tables.shape[1]), -1, dtype=np.int64)
+    for r, s in enumerate(seqs):
+        n = -(-lens[s] // 16)
+        bt[r, :n] = [remap[int(b)] for b in w.block_tables[s, :n]]
+    q = w.query[seqs].double().numpy()
+    nk = w.new_key[seqs].double().numpy()
+    nv = w.new_value[seqs].double().numpy()
+    sub_slots = [remap[int(slots[s]) // 16] * 16 + int(slots[s]) % 16 for s in seqs]
+    del kcv, vcv
+    info = threadpoolctl.threadpool_info()
+    threads = max([d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"] or [1])
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.reshape_and_cache(kc, vc, nk, nv, sub_slots, 16)
+        oracle.paged_decode(q, kc, vc, bt, [lens[s] for s in seqs], w.scale, w.num_kv_heads)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    kv = 2 * w.num_kv_heads * w.head_dim * 2 * sum(lens[s] for s in seqs) * reps
+    return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(seqs)} of {w.num_seqs} sequences (seeded), append + decode, "
+                      f"fp64 NumPy oracle, {reps} passes in {dt:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle on bounded samples of the same workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import threadpoolctl
+
+    import oracle
+    w = synth.llama3_8b_gqa_decode()
+    lens = (w.context_lens + 1).tolist()
+    rng = np.random.default_rng(1)
+    per_step = 8
+    info = threadpoolctl.threadpool_info()
+    threads = max([d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"] or [1])
+
+    def one_step(seqs):
+        used = sorted({int(b) for s in seqs for b in w.block_tables[s, :-(-lens[s] // 16)]})
+        remap = {b: i for i, b in enumerate(used)}
+        idx = torch.tensor(used)
+        kc = w.key_cache.index_select(0, idx).double().numpy()
+        vc = w.value_cache.index_select(0, idx).double().numpy()
+        bt = np.full((len(seqs), w.block_tables.shape[1]), -1, dtype=np.int64)
+        for r, s in enumerate(seqs):
+            n = -(-lens[s] // 16)
+            bt[r, :n] = [remap[int(b)] for b in w.block_tables[s, :n]]
+        q = w.query[seqs].double().numpy()
+        t0 = time.perf_counter()
+        sl = oracle.logical_positions_to_slots(bt, np.arange(len(seqs)),
+                                               w.context_lens[seqs].numpy(), 16)
+        oracle.reshape_and_cache(kc, vc, w.new_key[seqs].double().numpy(),
+                                 w.new_value[seqs].double().numpy(), sl, 16)
+        oracle.paged_decode(q, kc, vc, bt, [lens[s] for s in seqs], w.scale, w.num_kv_heads)
+        return time.perf_counter() - t0, 2 * w.num_kv_heads * w.head_dim * 2 * sum(
+            lens[s] for s in seqs)
+
+    for _ in range(args.warmup):
+        one_step(sorted(rng.choice(w.num_seqs, per_step, replace=False).tolist()))
+    tot_t = tot_b = 0.0
+    for _ in range(args.steps):
+        t, b = one_step(sorted(rng.choice(w.num_seqs, per_step, replace=False).tolist()))
+        tot_t += t
+        tot_b += b
+    value = tot_b / tot_t / 1e9
+    sample = f"{per_step} of {w.num_seqs} sequences per step (seeded), append + decode"
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--min-warmup-s", type=float, default=1.0,
+                    help="keep warming up for at least this long so clocks settle")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world, rank, local = setup_dist()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import paged_kv_cache_397_b200 as pa
+    pa.lib()
+
+    w = synth.llama3_8b_gqa_decode()
+    st = DecodeStep(w, dev)
+    stream = torch.cuda.current_stream()
+    hbm_peak, bf16_peak, peak_kind = peaks()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # warm-up: at least W steps and at least --min-warmup-s under load
+    t_end = time.time() + args.min_warmup_s
+    n = 0
+    while n < args.warmup or time.time() < t_end:
+        st.step()
+        n += 1
+    torch.cuda.synchronize()
+
+    # timed region: K full steps, plus per-launch events around pa_decode
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        st.append()
+        ev[i][0].record(stream)
+        st.decode()
+        ev[i][1].record(stream)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(t_start.elapsed_time(t_stop), world)
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    err = pa.pa_get_device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x} during the timed region")
+
+    ms_step = ms_total / args.steps
+    value = world * st.kv_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    achieved = st.kv_bytes / (decode_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(st.kv_bytes)
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    for _ in range(3):
+        st.step_e2e()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 200))
+    barrier(world)
+    e2e_ms = max_over_ranks(time_steps(st.step_e2e, e2e_steps, stream), world) / e2e_steps
+    e2e_value = world * st.kv_bytes / (e2e_ms * 1e-3) / 1e9
+
+    kv_bytes, launches = st.kv_bytes, st.launches_per_step * args.steps
+    h2d, d2h = st.h2d_bytes, st.d2h_bytes
+    prefill = None
+    if not args.no_prefill:
+        del st
+        torch.cuda.empty_cache()
+        prefill = []
+        for B in (16, 32):
+            r = prefill_measure(dev, steps=20, warmup=3, block_size=B)
+            r["tensor_frac"] = r["tflops"] / bf16_peak
+            r["peak_tflops"] = bf16_peak
+            r["peak_kind"] = f"bf16 dense, {peak_kind} (burst)"
+            prefill.append(r)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "kv_bytes_per_step_per_gpu": kv_bytes,
+                       "l2": "inputs larger than L2 (2.2 GB of K/V read per step, 126 MB L2)",
+                       "parallelism": f"replicas x{world} (each rank its own batch)"},
+            "hbm_frac": value / world / hbm_peak,
+            "decode_tokens_per_s": world * w.num_seqs / (ms_step * 1e-3),
+            "roofline": {"kernel": "pa_decode (decode_kernel + decode_reduce_kernel)",
+                         "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
+                         "peak_kind": f"hbm copy, {peak_kind}"},
+            "prefill_chunk": prefill,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,216 @@
+/*
+ * pa.h — C ABI of the B200 (sm_100a) paged-attention library (libpa.so).
+ *
+ * PagedAttention keeps each sequence's KV cache in fixed-size physical blocks
+ * of a shared pool and reaches them through a per-sequence block table that
+ * maps logical block i to a physical block anywhere in GPU memory
+ * ("vLLM PagedAttention Deep Dive", section "Virtual Memory Paging Analogy").
+ * Attention looks the blocks up, gathers K/V from them and runs standard
+ * attention, with a result identical to dense attention ("vLLM PagedAttention
+ * Deep Dive", section "PagedAttention Mechanism"; "PagedAttention: KV cache as
+ * virtual memory", section "Interviewer follow-ups").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  Layout.  key_cache and value_cache are separate pools, each a contiguous
+ *    T[num_blocks][num_kv_heads][block_size][head_dim] array (T = fp16 or
+ *    bf16).  A token at logical position p of sequence s lives in physical
+ *    block block_tables[s][p / block_size] at offset p % block_size; its slot
+ *    is physical_block * block_size + offset.
+ *  GQA.  Query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *  Pointers.  Every pointer argument is a DEVICE pointer, 16-byte aligned,
+ *    owned by the caller (the library allocates nothing and keeps no pointer
+ *    after a call returns).  Tensors are contiguous and row-major as stated.
+ *  Streams.  Every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  No call synchronises, except
+ *    pa_get_device_error.
+ *  Errors.  Host-side argument checks return PA_ERR_INVALID_ARG (null pointer,
+ *    non-positive or inconsistent size, misalignment) or PA_ERR_UNSUPPORTED
+ *    (a head_dim / block_size / dtype / group combination with no compiled
+ *    kernel) before anything is launched.  A failed launch returns
+ *    PA_ERR_CUDA.  Data-dependent errors found on the device (a slot or
+ *    physical block id outside [0, num_blocks), a sequence longer than its
+ *    block table, a bounded wait that ran out) never trap: the kernel records
+ *    a bit in a device error word, clamps or skips the offending access, and
+ *    carries on; pa_get_device_error reads and clears that word.
+ *  Block sizes 16 and 32; head_dim 64 and 128; query heads per KV head 1..16.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,
+  PA_ERR_UNSUPPORTED = 2,
+  PA_ERR_WORKSPACE = 3,
+  PA_ERR_OUT_OF_RANGE = 4,
+  PA_ERR_CUDA = 5
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word (pa_get_device_error). */
+#define PA_DEVERR_SLOT_RANGE 0x1u    /* slot_mapping entry >= num_blocks * block_size   */
+#define PA_DEVERR_BLOCK_RANGE 0x2u   /* block table / block pair id outside the pool    */
+#define PA_DEVERR_SEQ_RANGE 0x4u     /* sequence longer than max_blocks_per_seq blocks  */
+#define PA_DEVERR_WAIT_TIMEOUT 0x8u  /* a bounded barrier wait gave up                   */
+
+typedef struct CUstream_st *pa_stream_t; /* same type as cudaStream_t */
+
+/* Human-readable name of a pa_status value.  Never NULL. */
+const char *pa_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int pa_version(void);
+
+/*
+ * pa_slot_mapping — slot of every new token (logical position -> physical slot).
+ *   "vLLM PagedAttention Deep Dive", "PagedAttention Mechanism" (the block table
+ *   example) and "PagedAttention: KV cache as virtual memory", "Deep dive"
+ *   (tokens are appended at the end of the sequence).
+ * New token t belongs to sequence s with cu_q_lens[s] <= t < cu_q_lens[s+1]
+ * and sits at logical position ctx_lens[s] + (t - cu_q_lens[s]).  With
+ * cu_q_lens == NULL each sequence has exactly one new token (t == s, position
+ * ctx_lens[s]) and num_tokens must equal num_seqs.
+ *   slot_mapping  out  int64[num_tokens]
+ *   block_tables  in   int32[num_seqs][max_blocks_per_seq]
+ *   cu_q_lens     in   int32[num_seqs + 1] (non-decreasing, cu_q_lens[0] = 0,
+ *                      cu_q_lens[num_seqs] = num_tokens) or NULL
+ *   ctx_lens      in   int32[num_seqs]
+ * A position past the table (block index >= max_blocks_per_seq) yields slot -1
+ * and sets PA_DEVERR_SEQ_RANGE.
+ */
+pa_status pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
+                          const int32_t *cu_q_lens, const int32_t *ctx_lens, int num_seqs,
+                          int num_tokens, int max_blocks_per_seq, int block_size,
+                          pa_stream_t stream);
+
+/*
+ * pa_reshape_and_cache — scatter new tokens' K and V rows into their slots.
+ *   "PagedAttention: KV cache as virtual memory", "Deep dive" (the lifecycle:
+ *   decode takes one more block when the last one fills) and "PagedAttention:
+ *   Why Static Batching Wastes Your KV Cache", "What does PagedAttention
+ *   actually do differently?" (blocks are filled on demand).
+ * key_cache[slot / B][h][slot % B][:] = key[t][h][:] (same for value), a bit
+ * copy.  Slot -1 skips the token.  Slots must be distinct.
+ *   key, value              in      T[num_tokens][num_kv_heads][head_dim]
+ *   key_cache, value_cache  in/out  T[num_blocks][num_kv_heads][block_size][head_dim]
+ *   slot_mapping            in      int64[num_tokens]
+ * A slot >= num_blocks * block_size is skipped and sets PA_DEVERR_SLOT_RANGE.
+ */
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *key_cache,
+                               void *value_cache, const int64_t *slot_mapping, int num_tokens,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks — copy-on-write duplication of whole physical blocks.
+ *   "PagedAttention: Why Static Batching Wastes Your KV Cache", "How does
+ *   copy-on-write eliminate duplicate prompt KV cache?" (copy just that block
+ *   and remap the pointer, like fork()).
+ * For each pair (src, dst): key_cache[dst] = key_cache[src] and
+ * value_cache[dst] = value_cache[src] (all heads, slots and dims; bit copy).
+ * dst ids must be distinct and no dst may also be a src.
+ *   key_cache, value_cache  in/out  T[num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_pairs             in      int64[num_pairs][2] = {src, dst}
+ * A pair with an id outside [0, num_blocks) is skipped and sets PA_DEVERR_BLOCK_RANGE.
+ */
+pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *block_pairs,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_decode_partition_tokens — the split-KV partition length pa_decode uses
+ * for these sizes when called with partition_tokens == 0 (a multiple of
+ * block_size).  Host-only; touches no GPU.
+ */
+int pa_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_seq_len);
+
+/*
+ * pa_decode_workspace_size — bytes of scratch pa_decode needs for its split-KV
+ * partial results.  Host-only; touches no GPU.  partition_tokens as in
+ * pa_decode (0 = automatic).  Writes 0 when no sequence can span more than one
+ * partition.
+ */
+pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int max_seq_len, int partition_tokens,
+                                   size_t *bytes);
+
+/*
+ * pa_decode — one query token per sequence attending over its paged K/V.
+ *   "vLLM PagedAttention Deep Dive", "PagedAttention Mechanism" (look up the
+ *   physical blocks, gather K/V, standard attention) and "Chunked Prefill:
+ *   Preventing Compute Starvation" (decode is memory-bandwidth bound).
+ * out[s][h] = softmax(scale * q[s][h] . K_s^T) V_s over the first seq_lens[s]
+ * logical tokens of sequence s, K_s / V_s gathered through block_tables[s]
+ * for KV head h / G.  Long sequences are cut into partitions of
+ * partition_tokens tokens (0 = automatic); each partition's unnormalised
+ * softmax state goes to `workspace` and a second kernel combines them with a
+ * log-sum-exp reduction in a fixed order.  The arithmetic order depends only
+ * on logical positions, so the output is bit-identical under any relabelling
+ * of physical blocks.  seq_lens[s] == 0 gives a zero row.
+ *   out           out  T[num_seqs][num_q_heads][head_dim]
+ *   query         in   T[num_seqs][num_q_heads][head_dim]
+ *   key_cache, value_cache in T[num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_tables  in   int32[num_seqs][max_blocks_per_seq]; entries past
+ *                      ceil(seq_lens[s] / block_size) are never read
+ *   seq_lens      in   int32[num_seqs], each <= max_seq_len
+ *   max_seq_len   host upper bound of seq_lens (sizes the launch; no sync)
+ *   workspace     scratch of at least pa_decode_workspace_size bytes (may be
+ *                 NULL when that size is 0); returns PA_ERR_WORKSPACE if short
+ * A seq_len > max_blocks_per_seq * block_size sets PA_DEVERR_SEQ_RANGE (the
+ * extra tokens are ignored); a block id outside the pool is clamped to block
+ * 0 and sets PA_DEVERR_BLOCK_RANGE.
+ */
+pa_status pa_decode(void *out, const void *query, const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                    int partition_tokens, float scale, pa_dtype dtype, void *workspace,
+                    size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_prefill_chunk — causal chunked-prefill attention against the paged context.
+ *   "vLLM PagedAttention Deep Dive", "Mechanics of Chunked Prefill" (a long
+ *   prompt is processed chunk by chunk; each chunk's KV accumulates in paged
+ *   blocks) and "PagedAttention Mechanism".
+ * Sequence s has ctx_lens[s] tokens already cached and a chunk of
+ * n_s = cu_q_lens[s+1] - cu_q_lens[s] query tokens whose own K/V have already
+ * been written (pa_reshape_and_cache) at positions ctx_lens[s] .. ctx_lens[s]
+ * + n_s - 1.  Chunk query i (absolute position ctx_lens[s] + i) attends to
+ * positions 0 .. ctx_lens[s] + i inclusive.  Runs on the tcgen05 tensor cores
+ * (bf16/fp16 operands, fp32 accumulation in tensor memory).
+ *   out        out  T[total_q][num_q_heads][head_dim]
+ *   query      in   T[total_q][num_q_heads][head_dim]
+ *   cu_q_lens  in   int32[num_seqs + 1], cu_q_lens[num_seqs] == total_q
+ *   ctx_lens   in   int32[num_seqs]
+ *   max_q_len, max_ctx_len  host upper bounds (size the launch; no sync)
+ * head_dim must be 128.
+ */
+pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,
+                           const void *value_cache, const int32_t *block_tables,
+                           const int32_t *cu_q_lens, const int32_t *ctx_lens, int num_seqs,
+                           int total_q, int max_q_len, int max_ctx_len, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_blocks_per_seq, float scale, pa_dtype dtype,
+                           pa_stream_t stream);
+
+/*
+ * pa_get_device_error — synchronise `stream`, then read and clear the device
+ * error word of the current device (a bitwise OR of PA_DEVERR_* since the
+ * last read).  Returns PA_ERR_OUT_OF_RANGE when the word was non-zero.
+ */
+pa_status pa_get_device_error(unsigned int *error_word, pa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

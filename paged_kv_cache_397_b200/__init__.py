@@ -1,0 +1,249 @@
+"""Python binding of libpa.so, the B200 (sm_100a) paged-attention library.
+
+Argument marshalling only: every function takes torch CUDA tensors, checks
+their dtype / shape / contiguity, derives the sizes the C ABI wants from the
+shapes, and calls the ``extern "C"`` entry point of the same name in
+``libpa.so`` (declared in ``include/pa.h``) on the current CUDA stream.  Every
+step of the computation runs in the library's kernels; there is no CPU or
+PyTorch fallback — if ``libpa.so`` is missing, every call raises.
+
+Cited pages (by title and section): "vLLM PagedAttention Deep Dive: KV Cache
+Memory Fragmentation, Chunked Prefill & Prefix Caching" ("PagedAttention
+Mechanism", "Mechanics of Chunked Prefill"); "PagedAttention: KV cache as
+virtual memory" ("Deep dive"); "PagedAttention: Why Static Batching Wastes Your
+KV Cache" ("How does copy-on-write eliminate duplicate prompt KV cache?").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "PAError", "lib", "lib_path", "EXPORTED_SYMBOLS", "pa_status_string", "pa_version",
+    "pa_slot_mapping", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_partition_tokens",
+    "pa_decode_workspace_size", "pa_decode", "pa_prefill_chunk", "pa_get_device_error",
+    "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
+    "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16",
+    "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
+    "PA_DEVERR_WAIT_TIMEOUT",
+]
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = 0, 1, 2, 3
+PA_ERR_OUT_OF_RANGE, PA_ERR_CUDA = 4, 5
+PA_F16, PA_BF16 = 0, 1
+PA_DEVERR_SLOT_RANGE, PA_DEVERR_BLOCK_RANGE = 0x1, 0x2
+PA_DEVERR_SEQ_RANGE, PA_DEVERR_WAIT_TIMEOUT = 0x4, 0x8
+
+lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+
+# name -> (restype, argtypes); mirrors include/pa.h
+_i, _f, _p, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_SIGS = {
+    "pa_status_string": (ctypes.c_char_p, [_i]),
+    "pa_version": (_i, []),
+    "pa_slot_mapping": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p]),
+    "pa_reshape_and_cache": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]),
+    "pa_copy_blocks": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p]),
+    "pa_decode_partition_tokens": (_i, [_i, _i, _i, _i]),
+    "pa_decode_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
+    "pa_decode": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                       _p, _sz, _p]),
+    "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                              _i, _f, _i, _p]),
+    "pa_get_device_error": (_i, [ctypes.POINTER(ctypes.c_uint), _p]),
+}
+EXPORTED_SYMBOLS = tuple(_SIGS)
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+class PAError(RuntimeError):
+    """A libpa call returned a non-OK pa_status."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {pa_status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpa.so (once).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(
+                f"libpa.so not found at {lib_path}; build it with "
+                "`python -m paged_kv_cache_397_b200._build` (there is no CPU fallback)")
+        h = ctypes.CDLL(lib_path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = h
+    return _LIB
+
+
+def _check(fn: str, status: int) -> None:
+    if status != PA_OK:
+        raise PAError(fn, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+
+
+def _ptr(t, name: str, dtype=None, ndim=None) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _cache_dims(key_cache, value_cache):
+    if key_cache.shape != value_cache.shape or key_cache.dtype != value_cache.dtype:
+        raise ValueError("key_cache and value_cache must match in shape and dtype")
+    if key_cache.dim() != 4:
+        raise ValueError("caches must be [num_blocks][num_kv_heads][block_size][head_dim]")
+    return tuple(int(x) for x in key_cache.shape)
+
+
+def pa_status_string(status: int) -> str:
+    return lib().pa_status_string(int(status)).decode()
+
+
+def pa_version() -> int:
+    return lib().pa_version()
+
+
+def pa_slot_mapping(slot_mapping, block_tables, ctx_lens, block_size, cu_q_lens=None,
+                    stream=None):
+    """int64 slot of each new token (see include/pa.h, pa_slot_mapping)."""
+    S = int(ctx_lens.numel())
+    if block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("block_tables must be [num_seqs][max_blocks_per_seq]")
+    if cu_q_lens is not None and cu_q_lens.numel() != S + 1:
+        raise ValueError("cu_q_lens must have num_seqs + 1 entries")
+    _check("pa_slot_mapping", lib().pa_slot_mapping(
+        _ptr(slot_mapping, "slot_mapping", torch.int64, 1),
+        _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(cu_q_lens, "cu_q_lens", torch.int32, 1), _ptr(ctx_lens, "ctx_lens", torch.int32, 1),
+        S, int(slot_mapping.numel()), int(block_tables.shape[1]), int(block_size),
+        _stream(stream)))
+    return slot_mapping
+
+
+def pa_reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, stream=None):
+    """Scatter new K/V rows ``[num_tokens][num_kv_heads][head_dim]`` into their slots."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if key.shape != value.shape or key.dim() != 3 or tuple(key.shape[1:]) != (hkv, d):
+        raise ValueError("key/value must be [num_tokens][num_kv_heads][head_dim] like the cache")
+    if key.dtype != key_cache.dtype or value.dtype != key_cache.dtype:
+        raise ValueError("key/value dtype must match the cache")
+    if slot_mapping.numel() != key.shape[0]:
+        raise ValueError("slot_mapping needs one entry per token")
+    _check("pa_reshape_and_cache", lib().pa_reshape_and_cache(
+        _ptr(key, "key"), _ptr(value, "value"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(slot_mapping, "slot_mapping", torch.int64, 1),
+        int(key.shape[0]), hkv, d, bs, nb, _dtype_code(key_cache), _stream(stream)))
+
+
+def pa_copy_blocks(key_cache, value_cache, block_pairs, stream=None):
+    """Copy whole physical blocks: ``cache[dst] = cache[src]`` for each (src, dst) pair."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if block_pairs.dim() != 2 or block_pairs.shape[1] != 2:
+        raise ValueError("block_pairs must be int64 [num_pairs][2]")
+    _check("pa_copy_blocks", lib().pa_copy_blocks(
+        _ptr(key_cache, "key_cache"), _ptr(value_cache, "value_cache"),
+        _ptr(block_pairs, "block_pairs", torch.int64, 2), int(block_pairs.shape[0]), hkv, d, bs,
+        nb, _dtype_code(key_cache), _stream(stream)))
+
+
+def pa_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len) -> int:
+    return int(lib().pa_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len))
+
+
+def pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                             max_seq_len, partition_tokens=0) -> int:
+    n = ctypes.c_size_t(0)
+    _check("pa_decode_workspace_size", lib().pa_decode_workspace_size(
+        int(num_seqs), int(num_q_heads), int(num_kv_heads), int(head_dim), int(block_size),
+        int(max_seq_len), int(partition_tokens), ctypes.byref(n)))
+    return int(n.value)
+
+
+def pa_decode(out, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len, scale,
+              workspace=None, partition_tokens=0, stream=None):
+    """Paged decode attention: one query row per sequence (see include/pa.h, pa_decode).
+
+    ``workspace`` is a CUDA byte tensor of at least ``pa_decode_workspace_size``
+    bytes; when None the binding allocates one with torch.
+    """
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs][num_q_heads][head_dim]")
+    if query.dtype != key_cache.dtype or out.dtype != key_cache.dtype:
+        raise ValueError("query/out dtype must match the cache")
+    S, hq = int(query.shape[0]), int(query.shape[1])
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.numel() != S:
+        raise ValueError("block_tables / seq_lens do not match the batch")
+    need = pa_decode_workspace_size(S, hq, hkv, d, bs, max_seq_len, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode", lib().pa_decode(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(seq_lens, "seq_lens", torch.int32, 1), S, hq, hkv, d, bs, nb,
+        int(block_tables.shape[1]), int(max_seq_len), int(partition_tokens), float(scale),
+        _dtype_code(key_cache), ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def pa_prefill_chunk(out, query, key_cache, value_cache, block_tables, cu_q_lens, ctx_lens,
+                     max_q_len, max_ctx_len, scale, stream=None):
+    """Causal chunked-prefill attention against the paged context (include/pa.h)."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [total_q][num_q_heads][head_dim]")
+    if query.dtype != key_cache.dtype or out.dtype != key_cache.dtype:
+        raise ValueError("query/out dtype must match the cache")
+    S = int(ctx_lens.numel())
+    if cu_q_lens.numel() != S + 1 or block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("cu_q_lens / block_tables do not match ctx_lens")
+    _check("pa_prefill_chunk", lib().pa_prefill_chunk(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(cu_q_lens, "cu_q_lens", torch.int32, 1), _ptr(ctx_lens, "ctx_lens", torch.int32, 1),
+        S, int(query.shape[0]), int(max_q_len), int(max_ctx_len), int(query.shape[1]), hkv, d,
+        bs, nb, int(block_tables.shape[1]), float(scale), _dtype_code(key_cache),
+        _stream(stream)))
+    return out
+
+
+def pa_get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    w = ctypes.c_uint(0)
+    st = lib().pa_get_device_error(ctypes.byref(w), _stream(stream))
+    if st not in (PA_OK, PA_ERR_OUT_OF_RANGE):
+        raise PAError("pa_get_device_error", st)
+    return int(w.value)

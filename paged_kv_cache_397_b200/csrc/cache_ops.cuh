@@ -1,0 +1,107 @@
+// cache_ops.cuh — KV-cache writes for sm_100a: slot mapping, reshape_and_cache
+// (scatter new tokens into their slots) and copy_blocks (copy-on-write block
+// duplication).  All three are bit copies / integer work with 16-byte vector
+// accesses; at the sizes they run at (a few MB per call) they are bound by
+// launch latency and one HBM round trip, not by bandwidth.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace pa {
+
+// Slot of every new token: sequence s owns tokens [cu[s], cu[s+1]); token t
+// sits at logical position ctx_lens[s] + t - cu[s]; its slot is
+// block_tables[s][pos / B] * B + pos % B ("vLLM PagedAttention Deep Dive",
+// "PagedAttention Mechanism").  cu == nullptr: one token per sequence.
+__global__ void slot_mapping_kernel(int64_t* __restrict__ slots,
+                                    const int32_t* __restrict__ block_tables,
+                                    const int32_t* __restrict__ cu,
+                                    const int32_t* __restrict__ ctx_lens, int num_seqs,
+                                    int num_tokens, int max_blocks_per_seq, int block_size) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= num_tokens) return;
+  int s = t, off = 0;
+  if (cu != nullptr) {
+    // last s with cu[s] <= t (binary search over the non-decreasing offsets)
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(cu + mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+    off = t - __ldg(cu + s);
+  }
+  const int pos = __ldg(ctx_lens + s) + off;
+  const int blk = pos / block_size;
+  if (pos < 0 || blk >= max_blocks_per_seq) {
+    record_error(PA_DEVERR_SEQ_RANGE);
+    slots[t] = -1;
+    return;
+  }
+  const int phys = __ldg(block_tables + (size_t)s * max_blocks_per_seq + blk);
+  slots[t] = (int64_t)phys * block_size + (pos % block_size);
+}
+
+// One thread per 16-byte chunk of one (token, kv head) row of K and of V.
+template <int D>
+__global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
+                                         const uint4* __restrict__ value,
+                                         uint4* __restrict__ key_cache,
+                                         uint4* __restrict__ value_cache,
+                                         const int64_t* __restrict__ slot_mapping,
+                                         int num_tokens, int num_kv_heads, int block_size,
+                                         int64_t num_slots) {
+  constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)num_tokens * num_kv_heads * CH;
+  if (idx >= total) return;
+  const int c = (int)(idx % CH);
+  const int64_t th = idx / CH;  // token * Hkv + head
+  const int h = (int)(th % num_kv_heads);
+  const int64_t t = th / num_kv_heads;
+  const int64_t slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (c == 0) record_error(PA_DEVERR_SLOT_RANGE);
+    return;
+  }
+  const int64_t b = slot / block_size, off = slot % block_size;
+  const int64_t dst = ((b * num_kv_heads + h) * block_size + off) * CH + c;
+  const int64_t src = th * CH + c;
+  const uint4 kv = __ldg(key + src);
+  const uint4 vv = __ldg(value + src);
+  key_cache[dst] = kv;
+  value_cache[dst] = vv;
+}
+
+// One CTA per (pair, K-or-V); each thread moves kPerThread 16-byte chunks,
+// all loads issued before the stores.
+template <int kPerThread>
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
+                       const int64_t* __restrict__ pairs, int64_t chunks_per_block,
+                       int num_blocks) {
+  const int64_t src = __ldg(pairs + 2 * blockIdx.x), dst = __ldg(pairs + 2 * blockIdx.x + 1);
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0) record_error(PA_DEVERR_BLOCK_RANGE);
+    return;
+  }
+  uint4* cache = blockIdx.y == 0 ? key_cache : value_cache;
+  const uint4* from = cache + src * chunks_per_block;
+  uint4* to = cache + dst * chunks_per_block;
+  for (int64_t base = 0; base < chunks_per_block; base += (int64_t)kPerThread * 256) {
+    uint4 r[kPerThread];
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int64_t i = base + (int64_t)k * 256 + threadIdx.x;
+      if (i < chunks_per_block) r[k] = from[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int64_t i = base + (int64_t)k * 256 + threadIdx.x;
+      if (i < chunks_per_block) to[i] = r[k];
+    }
+  }
+}
+
+}  // namespace pa

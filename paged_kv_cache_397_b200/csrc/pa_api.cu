@@ -1,0 +1,376 @@
+// pa_api.cu — the extern "C" boundary of libpa.so (declared in include/pa.h):
+// argument validation, split-KV partition planning, TMA tensor-map encoding
+// and template dispatch onto the sm_100a kernels.  Nothing here allocates
+// device memory or synchronises (except pa_get_device_error).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <mutex>
+
+#include "../../include/pa.h"
+#include "cache_ops.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+constexpr int kVersion = (1 << 16) | 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library links no libcuda at build time and loads on machines without a GPU.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major [rows][cols] 16-bit tensor with a row pitch of `pitch_elems`,
+// boxes of {64 columns, box_rows rows}, 128-byte swizzle.
+bool make_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                 uint64_t pitch_elems, uint32_t box_rows, pa_dtype dt) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool valid_dtype(pa_dtype d) { return d == PA_F16 || d == PA_BF16; }
+
+// Split-KV partition length in tokens.  Partitions are whole blocks; the aim
+// is several waves of CTAs over 148 SMs while keeping each partition long
+// enough (>= 256 tokens) that its fixed cost and its partial write stay small.
+int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_seq_len) {
+  const long long units = (long long)num_seqs * num_kv_heads;
+  const long long target_ctas = 148LL * 3 * 8;  // ~8 waves at 3 CTAs per SM
+  long long per = (long long)max_seq_len * units / target_ctas;
+  int p = 256;
+  while (p < 2048 && p < per) p *= 2;
+  if (p < block_size) p = block_size;
+  return (p / block_size) * block_size;
+}
+
+int partition_tokens_for(int requested, int num_seqs, int num_kv_heads, int block_size,
+                         int max_seq_len) {
+  if (requested > 0) return ((requested + block_size - 1) / block_size) * block_size;
+  return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len);
+}
+
+template <typename T, int D, int BS, int NT>
+pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
+                     int num_parts, cudaStream_t stream) {
+  using Shape = pa::DecodeShape<T, D, BS, NT>;
+  auto kern = pa::decode_kernel<T, D, BS, NT>;
+  static bool configured = false;  // per instantiation; attribute is per device-function
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Shape::SMEM_BYTES) != cudaSuccess)
+      return PA_ERR_CUDA;
+    configured = true;
+  }
+  dim3 grid(num_parts, p.num_kv_heads, p.num_seqs);
+  kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (num_parts > 1) {
+    pa::decode_reduce_kernel<T, D><<<p.num_seqs * p.num_q_heads, D, 0, stream>>>(p, BS);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+template <typename T, int D, int BS>
+pa_status dispatch_group(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
+                         int num_parts, cudaStream_t stream) {
+  if (p.group <= 8) return run_decode<T, D, BS, 1>(mk, mv, p, num_parts, stream);
+  return run_decode<T, D, BS, 2>(mk, mv, p, num_parts, stream);
+}
+
+template <typename T>
+pa_status dispatch_decode(int D, int BS, const CUtensorMap& mk, const CUtensorMap& mv,
+                          pa::DecodeParams p, int num_parts, cudaStream_t stream) {
+  if (D == 128 && BS == 16) return dispatch_group<T, 128, 16>(mk, mv, p, num_parts, stream);
+  if (D == 128 && BS == 32) return dispatch_group<T, 128, 32>(mk, mv, p, num_parts, stream);
+  if (D == 64 && BS == 16) return dispatch_group<T, 64, 16>(mk, mv, p, num_parts, stream);
+  if (D == 64 && BS == 32) return dispatch_group<T, 64, 32>(mk, mv, p, num_parts, stream);
+  return PA_ERR_UNSUPPORTED;
+}
+
+template <typename T, int BS>
+pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      pa::PrefillParams p, int max_q_len, cudaStream_t stream) {
+  using Sh = pa::PrefillShape<T, BS>;
+  auto kern = pa::prefill_kernel<T, BS>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Sh::SMEM_BYTES) != cudaSuccess)
+      return PA_ERR_CUDA;
+    configured = true;
+  }
+  dim3 grid((max_q_len + Sh::BM - 1) / Sh::BM, p.num_q_heads, p.num_seqs);
+  kern<<<grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    case PA_ERR_OUT_OF_RANGE: return "PA_ERR_OUT_OF_RANGE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    default: return "PA_ERR_UNKNOWN";
+  }
+}
+
+int pa_version(void) { return kVersion; }
+
+pa_status pa_slot_mapping(int64_t* slot_mapping, const int32_t* block_tables,
+                          const int32_t* cu_q_lens, const int32_t* ctx_lens, int num_seqs,
+                          int num_tokens, int max_blocks_per_seq, int block_size,
+                          pa_stream_t stream) {
+  if (num_tokens < 0 || num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (num_seqs == 0 || !slot_mapping || !block_tables || !ctx_lens) return PA_ERR_INVALID_ARG;
+  if (cu_q_lens == nullptr && num_tokens != num_seqs) return PA_ERR_INVALID_ARG;
+  const int threads = 256;
+  pa::slot_mapping_kernel<<<(num_tokens + threads - 1) / threads, threads, 0,
+                            (cudaStream_t)stream>>>(slot_mapping, block_tables, cu_q_lens,
+                                                    ctx_lens, num_seqs, num_tokens,
+                                                    max_blocks_per_seq, block_size);
+  return launch_status();
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                               void* value_cache, const int64_t* slot_mapping, int num_tokens,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               pa_dtype dtype, pa_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  const long long total = (long long)num_tokens * num_kv_heads * (head_dim * 2 / 16);
+  const int threads = 256;
+  const long long grid = (total + threads - 1) / threads;
+  if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
+  const int64_t num_slots = (int64_t)num_blocks * block_size;
+  auto st = (cudaStream_t)stream;
+  auto k = reinterpret_cast<const uint4*>(key);
+  auto v = reinterpret_cast<const uint4*>(value);
+  auto kc = reinterpret_cast<uint4*>(key_cache);
+  auto vc = reinterpret_cast<uint4*>(value_cache);
+  if (head_dim == 128)
+    pa::reshape_and_cache_kernel<128><<<(unsigned)grid, threads, 0, st>>>(
+        k, v, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_slots);
+  else if (head_dim == 64)
+    pa::reshape_and_cache_kernel<64><<<(unsigned)grid, threads, 0, st>>>(
+        k, v, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_slots);
+  else
+    return PA_ERR_UNSUPPORTED;
+  return launch_status();
+}
+
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!key_cache || !value_cache || !block_pairs) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_INVALID_ARG;
+  if ((head_dim * 2) % 16 != 0) return PA_ERR_UNSUPPORTED;
+  const int64_t chunks = (int64_t)num_kv_heads * block_size * head_dim * 2 / 16;
+  pa::copy_blocks_kernel<8><<<dim3(num_pairs, 2), 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<uint4*>(key_cache), reinterpret_cast<uint4*>(value_cache), block_pairs,
+      chunks, num_blocks);
+  return launch_status();
+}
+
+int pa_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_seq_len) {
+  if (num_seqs <= 0 || num_kv_heads <= 0 || block_size <= 0 || max_seq_len < 0) return 0;
+  return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len);
+}
+
+pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int max_seq_len, int partition_tokens,
+                                   size_t* bytes) {
+  if (!bytes || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_seq_len < 0 || partition_tokens < 0)
+    return PA_ERR_INVALID_ARG;
+  const int pt = partition_tokens_for(partition_tokens, num_seqs, num_kv_heads, block_size,
+                                      max_seq_len);
+  const long long parts = max_seq_len == 0 ? 1 : ((long long)max_seq_len + pt - 1) / pt;
+  if (parts <= 1) {
+    *bytes = 0;
+    return PA_OK;
+  }
+  *bytes = (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * sizeof(float) + 256;
+  return PA_OK;
+}
+
+pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                    int partition_tokens, float scale, pa_dtype dtype, void* workspace,
+                    size_t workspace_bytes, pa_stream_t stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || max_seq_len < 0 || partition_tokens < 0 ||
+      !valid_dtype(dtype) || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if ((long long)max_seq_len > (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs > 65535) return PA_ERR_INVALID_ARG;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * num_kv_heads * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
+
+  const int pt = partition_tokens_for(partition_tokens, num_seqs, num_kv_heads, block_size,
+                                      max_seq_len);
+  const int num_parts = max_seq_len == 0 ? 1 : (max_seq_len + pt - 1) / pt;
+  if (num_parts > 65535) return PA_ERR_INVALID_ARG;
+  size_t need = 0;
+  pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                           max_seq_len, partition_tokens, &need);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return PA_ERR_WORKSPACE;
+
+  CUtensorMap mk, mv;
+  const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
+  if (!make_map_2d(&mk, key_cache, head_dim, rows, head_dim, block_size, dtype) ||
+      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, block_size, dtype))
+    return PA_ERR_CUDA;
+
+  pa::DecodeParams p;
+  p.out = out;
+  p.query = query;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  float* ws = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
+  const size_t acc_elems = (size_t)num_seqs * num_q_heads * num_parts * head_dim;
+  p.ws_acc = need > 0 ? ws : nullptr;
+  p.ws_ml = need > 0 ? ws + acc_elems : nullptr;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.num_blocks = num_blocks;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.part_blocks = pt / block_size;
+  p.max_parts = num_parts;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  auto st = (cudaStream_t)stream;
+  if (dtype == PA_BF16)
+    return dispatch_decode<__nv_bfloat16>(head_dim, block_size, mk, mv, p, num_parts, st);
+  return dispatch_decode<__half>(head_dim, block_size, mk, mv, p, num_parts, st);
+}
+
+pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
+                           const void* value_cache, const int32_t* block_tables,
+                           const int32_t* cu_q_lens, const int32_t* ctx_lens, int num_seqs,
+                           int total_q, int max_q_len, int max_ctx_len, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_blocks_per_seq, float scale, pa_dtype dtype,
+                           pa_stream_t stream) {
+  if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || max_ctx_len < 0 || num_q_heads <= 0 ||
+      num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || !valid_dtype(dtype) ||
+      !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || total_q == 0 || max_q_len == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !cu_q_lens || !ctx_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if ((long long)max_ctx_len >= (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs > 65535 || num_q_heads > 65535) return PA_ERR_INVALID_ARG;
+  if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * num_kv_heads * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
+  if ((long long)total_q * num_q_heads * head_dim > INT_MAX) return PA_ERR_INVALID_ARG;
+
+  CUtensorMap mq, mk, mv;
+  const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
+  if (!make_map_2d(&mq, query, (uint64_t)num_q_heads * head_dim, total_q,
+                   (uint64_t)num_q_heads * head_dim, 128, dtype) ||
+      !make_map_2d(&mk, key_cache, head_dim, rows, head_dim, block_size, dtype) ||
+      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, block_size, dtype))
+    return PA_ERR_CUDA;
+  pa::PrefillParams p;
+  p.out = out;
+  p.block_tables = block_tables;
+  p.cu_q_lens = cu_q_lens;
+  p.ctx_lens = ctx_lens;
+  p.num_seqs = num_seqs;
+  p.total_q = total_q;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.num_blocks = num_blocks;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  auto st = (cudaStream_t)stream;
+  if (dtype == PA_BF16) {
+    if (block_size == 16) return run_prefill<__nv_bfloat16, 16>(mq, mk, mv, p, max_q_len, st);
+    return run_prefill<__nv_bfloat16, 32>(mq, mk, mv, p, max_q_len, st);
+  }
+  if (block_size == 16) return run_prefill<__half, 16>(mq, mk, mv, p, max_q_len, st);
+  return run_prefill<__half, 32>(mq, mk, mv, p, max_q_len, st);
+}
+
+pa_status pa_get_device_error(unsigned int* error_word, pa_stream_t stream) {
+  if (!error_word) return PA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_error_word, sizeof(v)) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return PA_ERR_CUDA;
+  *error_word = v;
+  return v == 0 ? PA_OK : PA_ERR_OUT_OF_RANGE;
+}
+
+}  // extern "C"
