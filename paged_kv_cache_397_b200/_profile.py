@@ -1,0 +1,76 @@
+"""Small, self-contained cases of the hot kernels for ncu captures.
+
+    python -m paged_kv_cache_397_b200._profile decode  --seqs 32
+    python -m paged_kv_cache_397_b200._profile prefill --seqs 4 [--block-size 16]
+
+Each case builds a scaled-down copy of a bench workload (same shapes, head
+counts, length distribution and block shuffling; fewer sequences), runs the
+kernel three times on cuda:0 and prints the launch's K/V bytes or FLOPs, so
+per-launch counters can be scaled to the full-size launch.  The inputs stay a
+few hundred MB on the device (above the 126 MB L2) so that a multi-pass
+capture ends in seconds.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import paged_kv_cache_397_b200 as pa  # noqa: E402
+import synth  # noqa: E402
+
+
+def decode_case(seqs: int, reps: int = 3):
+    w = synth.llama3_8b_gqa_decode(num_seqs=seqs)
+    d = torch.device("cuda:0")
+    kc, vc, bt = w.key_cache.to(d), w.value_cache.to(d), w.block_tables.to(d)
+    lens = (w.context_lens + 1).to(d)
+    q = w.query.to(d)
+    out = torch.empty_like(q)
+    max_len = int(lens.max())
+    for _ in range(reps):
+        pa.pa_decode(out, q, kc, vc, bt, lens, max_len, w.scale)
+    torch.cuda.synchronize()
+    kv = 2 * w.num_kv_heads * w.head_dim * 2 * int(lens.sum())
+    print(f"decode case: {w.name}, K/V bytes per launch {kv}")
+
+
+def prefill_case(seqs: int, block_size: int, reps: int = 3):
+    p = synth.chunked_prefill(num_seqs=seqs, block_size=block_size)
+    d = torch.device("cuda:0")
+    kc, vc = p.key_cache.to(d), p.value_cache.to(d)
+    bt, cl, cu = p.block_tables.to(d), p.ctx_lens.to(d), p.cu_q_lens.to(d)
+    q = p.query.to(d)
+    out = torch.empty_like(q)
+    qmax, cmax = int(torch.diff(p.cu_q_lens).max()), int(p.ctx_lens.max())
+    for _ in range(reps):
+        pa.pa_prefill_chunk(out, q, kc, vc, bt, cu, cl, qmax, cmax, p.scale)
+    torch.cuda.synchronize()
+    flops = sum(4 * p.head_dim * p.num_q_heads * (n * c + n * (n + 1) // 2)
+                for c, n in zip(p.ctx_lens.tolist(), torch.diff(p.cu_q_lens).tolist()))
+    print(f"prefill case: {p.name}, causal FLOP per launch {flops}")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["decode", "prefill"])
+    ap.add_argument("--seqs", type=int, default=None)
+    ap.add_argument("--block-size", type=int, default=16)
+    a = ap.parse_args()
+    pa.lib()
+    if a.case == "decode":
+        decode_case(a.seqs or 32)
+    else:
+        prefill_case(a.seqs or 4, a.block_size)
+    if pa.pa_get_device_error():
+        raise SystemExit("device error word set")
+
+
+if __name__ == "__main__":
+    main()
