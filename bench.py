@@ -143,11 +143,18 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time (all ranks call this in the same order)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job GB/s: the bytes every rank processed over the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / 1e9
 
 
 class DecodeStep:
@@ -409,7 +416,7 @@ def main():
         raise RuntimeError(f"device error word {err:#x} during the timed region")
 
     ms_step = ms_total / args.steps
-    value = world * st.kv_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    value = job_throughput(st.kv_bytes, world, args.steps, ms_total)
     achieved = st.kv_bytes / (decode_ms * 1e-3) / 1e9
     traffic = profiled_traffic(st.kv_bytes)
 
@@ -420,7 +427,7 @@ def main():
     e2e_steps = max(3, min(args.steps, 200))
     barrier(world)
     e2e_ms = max_over_ranks(time_steps(st.step_e2e, e2e_steps, stream), world) / e2e_steps
-    e2e_value = world * st.kv_bytes / (e2e_ms * 1e-3) / 1e9
+    e2e_value = job_throughput(st.kv_bytes, world, 1, e2e_ms)
 
     kv_bytes, launches = st.kv_bytes, st.launches_per_step * args.steps
     h2d, d2h = st.h2d_bytes, st.d2h_bytes
