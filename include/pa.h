@@ -177,6 +177,39 @@ pa_status pa_decode(void *out, const void *query, const void *key_cache, const v
                     size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_decode_static_workspace — pa_decode for callers that cannot allocate
+ * device memory.  (No counterpart on the pages: this is a library service,
+ * not part of the paged-attention method.)
+ * Some callers cannot call cudaMalloc: for example a plugin running inside an
+ * inference runtime that owns and budgets all device memory itself, or a
+ * latency-critical serving loop that must not allocate after start-up (an
+ * allocation can synchronise the device and can fail under memory pressure).
+ * This entry point takes the same arguments as pa_decode minus the
+ * workspace: its split-KV scratch lives in one file-scope device array of
+ * PA_STATIC_WORKSPACE_BYTES bytes that every GPU which loads the library
+ * holds until the process exits.  It allocates nothing itself.
+ *   - Requests whose pa_decode_workspace_size exceeds
+ *     PA_STATIC_WORKSPACE_BYTES return PA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device (with that device current) resolves the
+ *     array's device address with cudaGetSymbolAddress and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array, and it keeps the last
+ *     call's contents.  The decode kernels write every partial result before
+ *     they read it, so nothing needs clearing; but calls that overlap on the
+ *     GPU (e.g. on two streams at once) race on the array and must be
+ *     serialised by the caller.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+pa_status pa_decode_static_workspace(void *out, const void *query, const void *key_cache,
+                                     const void *value_cache, const int32_t *block_tables,
+                                     const int32_t *seq_lens, int num_seqs, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                                     int partition_tokens, float scale, pa_dtype dtype,
+                                     pa_stream_t stream);
+
+/*
  * pa_prefill_chunk — causal chunked-prefill attention against the paged context.
  *   "vLLM PagedAttention Deep Dive", "Mechanics of Chunked Prefill" (a long
  *   prompt is processed chunk by chunk; each chunk's KV accumulates in paged

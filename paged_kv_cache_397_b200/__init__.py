@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "PAError", "lib", "lib_path", "EXPORTED_SYMBOLS", "pa_status_string", "pa_version",
     "pa_slot_mapping", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_partition_tokens",
-    "pa_decode_workspace_size", "pa_decode", "pa_prefill_chunk", "pa_get_device_error",
+    "pa_decode_workspace_size", "pa_decode", "pa_decode_static_workspace", "pa_prefill_chunk",
+    "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
@@ -51,6 +52,8 @@ _SIGS = {
     "pa_decode_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "pa_decode": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
                        _p, _sz, _p]),
+    "pa_decode_static_workspace": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                                        _i, _i, _f, _i, _p]),
     "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                               _i, _f, _i, _p]),
     "pa_get_device_error": (_i, [ctypes.POINTER(ctypes.c_uint), _p]),
@@ -216,6 +219,35 @@ def pa_decode(out, query, key_cache, value_cache, block_tables, seq_lens, max_se
         _ptr(seq_lens, "seq_lens", torch.int32, 1), S, hq, hkv, d, bs, nb,
         int(block_tables.shape[1]), int(max_seq_len), int(partition_tokens), float(scale),
         _dtype_code(key_cache), ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+PA_STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def pa_decode_static_workspace(out, query, key_cache, value_cache, block_tables, seq_lens,
+                               max_seq_len, scale, partition_tokens=0, stream=None):
+    """pa_decode with its scratch in the library's own per-device array.
+
+    For callers that must not allocate device memory (see include/pa.h): no
+    workspace argument, nothing allocated here or in the library.  Requests
+    needing more than PA_STATIC_WORKSPACE_BYTES of scratch raise PAError
+    (PA_ERR_WORKSPACE); concurrent calls on one device must be serialised.
+    """
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs][num_q_heads][head_dim]")
+    if query.dtype != key_cache.dtype or out.dtype != key_cache.dtype:
+        raise ValueError("query/out dtype must match the cache")
+    S, hq = int(query.shape[0]), int(query.shape[1])
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.numel() != S:
+        raise ValueError("block_tables / seq_lens do not match the batch")
+    _check("pa_decode_static_workspace", lib().pa_decode_static_workspace(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(seq_lens, "seq_lens", torch.int32, 1), S, hq, hkv, d, bs, nb,
+        int(block_tables.shape[1]), int(max_seq_len), int(partition_tokens), float(scale),
+        _dtype_code(key_cache), _stream(stream)))
     return out
 
 

@@ -61,6 +61,31 @@ bool make_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 
 bool valid_dtype(pa_dtype d) { return d == PA_F16 || d == PA_BF16; }
 
+// Split-KV scratch for pa_decode_static_workspace, for callers that cannot
+// allocate: one array per device, part of the module's own device memory.
+// Host code must not pass the symbol itself to a kernel (on the host it is a
+// stand-in, not a device address); static_workspace_address resolves the real
+// address once per device, with that device current, and caches it.
+static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_addr[kMaxDevices] = {};
+
+pa_status static_workspace_address(void** addr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (g_static_ws_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
+      return PA_ERR_CUDA;
+    g_static_ws_addr[dev] = p;
+  }
+  *addr = g_static_ws_addr[dev];
+  return PA_OK;
+}
+
 // Split-KV partition length in tokens.  Partitions are whole blocks; the aim
 // is several waves of CTAs over 148 SMs while keeping each partition long
 // enough (>= 256 tokens) that its fixed cost and its partial write stay small.
@@ -306,6 +331,29 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
   if (dtype == PA_BF16)
     return dispatch_decode<__nv_bfloat16>(head_dim, block_size, mk, mv, p, num_parts, st);
   return dispatch_decode<__half>(head_dim, block_size, mk, mv, p, num_parts, st);
+}
+
+pa_status pa_decode_static_workspace(void* out, const void* query, const void* key_cache,
+                                     const void* value_cache, const int32_t* block_tables,
+                                     const int32_t* seq_lens, int num_seqs, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                                     int partition_tokens, float scale, pa_dtype dtype,
+                                     pa_stream_t stream) {
+  size_t need = 0;
+  pa_status st = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                          block_size, max_seq_len, partition_tokens, &need);
+  if (st != PA_OK) return st;
+  if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    st = static_workspace_address(&ws);
+    if (st != PA_OK) return st;
+  }
+  return pa_decode(out, query, key_cache, value_cache, block_tables, seq_lens, num_seqs,
+                   num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                   max_blocks_per_seq, max_seq_len, partition_tokens, scale, dtype, ws,
+                   need > 0 ? (size_t)PA_STATIC_WORKSPACE_BYTES : 0, stream);
 }
 
 pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
