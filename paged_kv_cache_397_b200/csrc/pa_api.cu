@@ -156,7 +156,8 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
       return PA_ERR_CUDA;
     configured = true;
   }
-  dim3 grid((max_q_len + Sh::BM - 1) / Sh::BM, p.num_q_heads, p.num_seqs);
+  constexpr int rows_per_cta = Sh::NQ * Sh::BM;
+  dim3 grid((max_q_len + rows_per_cta - 1) / rows_per_cta, p.num_q_heads, p.num_seqs);
   kern<<<grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return launch_status();
 }

@@ -7,25 +7,31 @@
 // attention, to the logical tokens 0 .. ctx_lens[s] + i of its KV head, read
 // through block_tables[s]; the chunk's own K/V are already in the cache.
 //
-// How (B200 design, one CTA per (128-query tile, query head, sequence)):
-//  * warp 4 (TMA): loads the Q tile once and streams 128-token K and V tiles
-//    into a 2-stage ring.  A tile is gathered block by block: each logical
-//    block is one TMA box per 64 columns at row (phys * Hkv + kvh) * B of the
-//    pool viewed as a 2-D [rows, head_dim] tensor, 128-byte swizzled, so the
-//    gather needs no address arithmetic on the compute warps.
-//  * warp 5 (MMA, one thread): S_j = Q K_j^T with tcgen05.mma (M=128, N=128,
-//    K=16 steps, both operands K-major in shared memory) into one of two
-//    128-column TMEM buffers; then O += P_{j-1} V_{j-1} with P read from
-//    tensor memory and V as an MN-major shared-memory operand.  Completion is
-//    signalled with tcgen05.commit on mbarriers.
-//  * warps 0-3 (softmax): thread r owns query row r = TMEM lane r.  It loads
-//    its S row with tcgen05.ld, applies the causal / length mask, keeps a
-//    running max that is only raised when the tile max exceeds it by more
-//    than 2^8 (so O is rescaled in TMEM rarely; the stale max cancels in
-//    O / l), writes P = exp2(S - m) as 16-bit values over the S buffer with
-//    tcgen05.st, and finally divides O by the row sum and stores the row.
+// How (B200 design).  One CTA per (256 chunk rows, query head, sequence); the
+// 256 rows are two 128-row Q tiles that share every K/V tile:
+//  * warp 8 (TMA): loads both Q tiles once, then streams K_0, V_0, K_1, V_1,
+//    ... through a 4-stage shared-memory ring.  A 128-token tile is gathered
+//    block by block — one TMA box per block per 64 columns at row
+//    (phys * Hkv + kvh) * B of the pool viewed as a 2-D [rows, head_dim]
+//    tensor, 128-byte swizzled — with the boxes of a tile issued in parallel
+//    by the warp's lanes.
+//  * warp 9 (MMA, one thread): tcgen05.mma kind::f16, fp32 accumulation in
+//    tensor memory.  S_w = Q_w K_j^T (M=128, N=128, K-major operands in
+//    shared memory) and O_w += P_w V_j (P from tensor memory, V an MN-major
+//    shared-memory operand).  Issue order: S0_0, S1_0, then for every tile
+//    PV0_j, S0_{j+1}, PV1_j, S1_{j+1}: while one softmax warpgroup works on
+//    its scores, the tensor core runs the other tile's products.
+//    Completion is signalled with tcgen05.commit on mbarriers.
+//  * warps 0-3 and 4-7 (softmax, one warpgroup per Q tile): thread r owns
+//    query row r = TMEM lane r.  It loads its S row (tcgen05.ld), masks only
+//    on tiles that reach past its causal limit, keeps a running max raised
+//    only when a tile's max exceeds it by more than 2^8 (the stale max
+//    cancels in O / l, so O in tensor memory is rarely rescaled), writes
+//    P = exp2(S * scale - m) as 16-bit values over its S columns (tcgen05.st),
+//    and finally stores O / l.  Because S_w(j) is issued after PV_w(j-1),
+//    "S_w(j) complete" already implies O_w is up to date for a rescale.
 //  * V rows past the end of the sequence (unwritten slots, NaN allowed) are
-//    zeroed in shared memory before their PV product.
+//    zeroed in shared memory by warpgroup 0 before the last PV products.
 #pragma once
 
 #include <type_traits>
@@ -47,20 +53,47 @@ struct PrefillParams {
 template <typename T, int BS>
 struct PrefillShape {
   static constexpr int D = 128;
-  static constexpr int BM = 128;                // query rows per CTA
-  static constexpr int BN = 128;                // keys per tile
-  static constexpr int THREADS = 6 * 32;
-  static constexpr int HALF = BM * 128;         // one 64-column group of a 128-row tile (16 KB)
+  static constexpr int BM = 128;                // rows per Q tile
+  static constexpr int NQ = 2;                  // Q tiles per CTA
+  static constexpr int BN = 128;                // keys per K/V tile
+  static constexpr int THREADS = 10 * 32;
+  static constexpr int TMA_WARP = 8, MMA_WARP = 9;
+  static constexpr int HALF = 128 * 128;        // 128 rows x 64 columns x 2 bytes
   static constexpr int TILE = 2 * HALF;         // 128 x 128 x 2 bytes = 32 KB
+  static constexpr int NSTAGE = 4;              // K/V ring stages (K_j, V_j alternate)
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE;            // 2 stages
-  static constexpr int V_OFF = 3 * TILE;        // 2 stages
-  static constexpr int BAR_OFF = 5 * TILE;
-  static constexpr int NBAR = 16;
+  static constexpr int RING_OFF = NQ * TILE;
+  static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE;
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 3 * NQ;
   static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBAR * 8 + 16;
   static constexpr int BLOCKS_PER_TILE = BN / BS;
-  static constexpr uint32_t TMEM_COLS = 512;    // S0 | S1 | O | (unused)
+  static constexpr uint32_t TMEM_COLS = 512;    // S0 | S1 | O0 | O1
+  static_assert(2 * BLOCKS_PER_TILE <= 32, "one TMA box per lane");
 };
+
+// S_w = Q_w K^T: 8 K-steps of 16 over head_dim, both operands K-major, SW128.
+template <int HALF>
+__device__ __forceinline__ void prefill_issue_s(uint32_t d_tmem, uint32_t q_smem,
+                                                uint32_t k_smem, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+    umma_ss(d_tmem, umma_desc_sw128(q_smem + off, 16, 1024),
+            umma_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+  }
+}
+
+// O_w += P_w V: 8 K-steps of 16 keys; P from tensor memory (8 columns of
+// packed 16-bit pairs per step), V MN-major with its two 64-column halves
+// HALF bytes apart.
+template <int HALF>
+__device__ __forceinline__ void prefill_issue_pv(uint32_t o_tmem, uint32_t p_tmem,
+                                                 uint32_t v_smem, uint32_t idesc, bool first) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_ts(o_tmem, p_tmem + kk * 8, umma_desc_sw128(v_smem + kk * 16 * 128, HALF, 1024), idesc,
+            (!first || kk > 0) ? 1u : 0u);
+}
 
 template <typename T, int BS>
 __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
@@ -68,54 +101,49 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
   using Sh = PrefillShape<T, BS>;
-  constexpr int D = Sh::D, BM = Sh::BM, BN = Sh::BN;
+  constexpr int D = Sh::D, BM = Sh::BM, BN = Sh::BN, NQ = Sh::NQ, NS = Sh::NSTAGE;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::BAR_OFF);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* p_full = bars + 11;  // [2]
-  uint64_t* o_done = bars + 13;
-  uint64_t* o_final = bars + 14;
+  uint64_t* q_full = bars;                        // 1
+  uint64_t* ring_full = bars + 1;                 // NS
+  uint64_t* ring_empty = bars + 1 + NS;           // NS
+  uint64_t* s_full = bars + 1 + 2 * NS;           // NQ
+  uint64_t* p_full = s_full + NQ;                 // NQ
+  uint64_t* o_final = p_full + NQ;                // NQ
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Sh::NBAR);
 
-  const int qtile = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int h = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = p.cu_q_lens[s];
   const int n = p.cu_q_lens[s + 1] - q0;
-  const int i0 = qtile * BM;
+  const int i0 = blockIdx.x * (NQ * BM);  // first chunk row of this CTA
   if (i0 >= n) return;
   const int c = p.ctx_lens[s];
   int L = c + n;  // tokens in the cache for this sequence
   if (L > p.max_blocks_per_seq * BS) {
-    if (threadIdx.x == 0 && h == 0 && qtile == 0) record_error(PA_DEVERR_SEQ_RANGE);
+    if (threadIdx.x == 0 && h == 0 && blockIdx.x == 0) record_error(PA_DEVERR_SEQ_RANGE);
     L = p.max_blocks_per_seq * BS;
   }
   const int kvh = h / p.group;
-  const int rows = min(BM, n - i0);
-  // keys needed by the last row of this tile (bounded by the sequence length)
-  const int kv_end = min(L, c + i0 + rows);
-  const int ntiles = (kv_end + BN - 1) / BN;
+  const int rows = min(NQ * BM, n - i0);            // valid rows of this CTA
+  const int kv_end = min(L, c + i0 + rows);         // keys the last valid row needs
+  const int ntiles = (kv_end + BN - 1) / BN;        // >= 1
   const int nblk_seq = (L + BS - 1) / BS;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
+    for (int w = 0; w < NQ; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], 128);
+      mbar_init(&o_final[w], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -126,10 +154,8 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s[2] = {tmem, tmem + 128};
-  const uint32_t t_o = tmem + 256;
 
-  if (warp == 4) {
+  if (warp == Sh::TMA_WARP) {
     // ------------------------------------------------------------ TMA warp
     const uint64_t pol_kv = l2_policy_evict_last();
     const uint64_t pol_q = l2_policy_evict_first();
@@ -137,15 +163,17 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(q_full, Sh::TILE);
-      for (int hf = 0; hf < 2; ++hf)
-        tma_load_2d(smem + Sh::Q_OFF + hf * Sh::HALF, &tm_q, h * D + hf * 64, q0 + i0, q_full,
-                    pol_q);
+      mbar_arrive_expect_tx(q_full, NQ * Sh::TILE);
+    }
+    __syncwarp();
+    if (lane < 2 * NQ) {  // lane -> (Q tile, 64-column half)
+      const int w = lane >> 1, hf = lane & 1;
+      tma_load_2d(smem + Sh::Q_OFF + w * Sh::TILE + hf * Sh::HALF, &tm_q, h * D + hf * 64,
+                  q0 + i0 + w * BM, q_full, pol_q);
     }
     const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq;
     bool alive = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
       const int b0 = j * Sh::BLOCKS_PER_TILE;
       const int nb = min(Sh::BLOCKS_PER_TILE, nblk_seq - b0);
       int phys = 0;
@@ -156,176 +184,182 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
           phys = 0;
         }
       }
+      // lane l issues the box of block l / 2, 64-column half l % 2
+      const int ph = __shfl_sync(0xffffffffu, phys, (lane >> 1) & 31);
+      const int row = (ph * p.num_kv_heads + kvh) * BS;
       const uint32_t bytes = (uint32_t)nb * BS * D * 2;
-      if (lane == 0) {
-        if (j >= 2 && alive) alive = mbar_wait(&k_empty[st], ((j >> 1) - 1) & 1);
-        mbar_arrive_expect_tx(&k_full[st], bytes);
-      }
-      for (int b = 0; b < nb; ++b) {
-        const int ph = __shfl_sync(0xffffffffu, phys, b);
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const int item = 2 * j + kv, st = item % NS;
         if (lane == 0) {
-          const int row = (ph * p.num_kv_heads + kvh) * BS;
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d(smem + Sh::K_OFF + st * Sh::TILE + hf * Sh::HALF + b * BS * 128, &tm_k,
-                        hf * 64, row, &k_full[st], pol_kv);
+          if (item >= NS && alive) alive = mbar_wait(&ring_empty[st], ((item / NS) - 1) & 1);
+          mbar_arrive_expect_tx(&ring_full[st], bytes);
         }
-      }
-      if (lane == 0) {
-        if (j >= 2 && alive) alive = mbar_wait(&v_empty[st], ((j >> 1) - 1) & 1);
-        mbar_arrive_expect_tx(&v_full[st], bytes);
-      }
-      for (int b = 0; b < nb; ++b) {
-        const int ph = __shfl_sync(0xffffffffu, phys, b);
-        if (lane == 0) {
-          const int row = (ph * p.num_kv_heads + kvh) * BS;
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d(smem + Sh::V_OFF + st * Sh::TILE + hf * Sh::HALF + b * BS * 128, &tm_v,
-                        hf * 64, row, &v_full[st], pol_kv);
+        __syncwarp();
+        if (lane < 2 * nb) {
+          tma_load_2d(smem + Sh::RING_OFF + st * Sh::TILE + (lane & 1) * Sh::HALF +
+                          (lane >> 1) * BS * 128,
+                      kv == 0 ? &tm_k : &tm_v, (lane & 1) * 64, row, &ring_full[st], pol_kv);
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == Sh::MMA_WARP) {
     // ------------------------------------------------------------ MMA warp
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_f16(128, 128, kBf16, false, false);
       constexpr uint32_t idesc_pv = umma_idesc_f16(128, 128, kBf16, false, true);
       const uint32_t sq = smem_u32(smem + Sh::Q_OFF);
+      const uint32_t ring = smem_u32(smem + Sh::RING_OFF);
       bool alive = mbar_wait(q_full, 0);
+      if (alive) alive = mbar_wait(&ring_full[0], 0);  // K_0
       tc_fence_after();
-      for (int j = 0; j <= ntiles; ++j) {
-        if (j < ntiles) {
-          const int st = j & 1;
-          if (alive) alive = mbar_wait(&k_full[st], (j >> 1) & 1);
+      prefill_issue_s<Sh::HALF>(tmem, sq, ring, idesc_qk);
+      umma_commit(&s_full[0]);
+      prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring, idesc_qk);
+      umma_commit(&s_full[1]);
+      umma_commit(&ring_empty[0]);
+      for (int j = 0; j < ntiles; ++j) {
+        const int it_v = 2 * j + 1, st_v = it_v % NS;
+        const int it_k = 2 * j + 2, st_k = it_k % NS;
+        const bool more = j + 1 < ntiles;
+        // tile 0: PV0_j, then S0_{j+1}
+        if (alive) alive = mbar_wait(&p_full[0], j & 1);
+        if (alive) alive = mbar_wait(&ring_full[st_v], (it_v / NS) & 1);
+        tc_fence_after();
+        prefill_issue_pv<Sh::HALF>(tmem + 256, tmem, ring + st_v * Sh::TILE, idesc_pv, j == 0);
+        if (more) {
+          if (alive) alive = mbar_wait(&ring_full[st_k], (it_k / NS) & 1);
           tc_fence_after();
-          const uint32_t sk = smem_u32(smem + Sh::K_OFF + st * Sh::TILE);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * Sh::HALF + (kk & 3) * 32;
-            umma_ss(t_s[st], umma_desc_sw128(sq + off, 16, 1024),
-                    umma_desc_sw128(sk + off, 16, 1024), idesc_qk, kk > 0);
-          }
-          umma_commit(&s_full[st]);
-          umma_commit(&k_empty[st]);
+          prefill_issue_s<Sh::HALF>(tmem, sq, ring + st_k * Sh::TILE, idesc_qk);
+          umma_commit(&s_full[0]);
+        } else {
+          umma_commit(&o_final[0]);
         }
-        if (j >= 1) {
-          const int jp = j - 1, st = jp & 1;
-          if (alive) alive = mbar_wait(&p_full[st], (jp >> 1) & 1);
-          if (alive) alive = mbar_wait(&v_full[st], (jp >> 1) & 1);
-          tc_fence_after();
-          const uint32_t sv = smem_u32(smem + Sh::V_OFF + st * Sh::TILE);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            umma_ts(t_o, t_s[st] + kk * 8, umma_desc_sw128(sv + kk * 16 * 128, Sh::HALF, 1024),
-                    idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&v_empty[st]);
-          umma_commit(o_done);
-          if (j == ntiles) umma_commit(o_final);
+        // tile 1: PV1_j, then S1_{j+1}
+        if (alive) alive = mbar_wait(&p_full[1], j & 1);
+        tc_fence_after();
+        prefill_issue_pv<Sh::HALF>(tmem + 384, tmem + 128, ring + st_v * Sh::TILE, idesc_pv,
+                                   j == 0);
+        umma_commit(&ring_empty[st_v]);
+        if (more) {
+          prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring + st_k * Sh::TILE, idesc_qk);
+          umma_commit(&s_full[1]);
+          umma_commit(&ring_empty[st_k]);
+        } else {
+          umma_commit(&o_final[1]);
         }
       }
     }
   } else {
-    // -------------------------------------------------------- softmax warps
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int qpos = c + i0 + r;                // absolute position of this row's query
-    const int limit = min(qpos, L - 1);         // last visible key
-    float m_run = -INFINITY, l_run = 0.f;
+    // -------------------------------------------------- softmax warpgroups
+    const int w = warp >> 2;                       // Q tile of this warpgroup
+    const int r = threadIdx.x & 127;               // row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + w * 128;
+    const uint32_t t_o = tmem + lane_base + 256 + w * 128;
+    const int row = i0 + w * BM + r;               // chunk row of this thread
+    const int limit = min(c + row, L - 1);         // last key this row may see
+    const float sc = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;          // running max in log2 units
     bool alive = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
-      if (alive) alive = mbar_wait(&s_full[st], (j >> 1) & 1);
+      if (alive) alive = mbar_wait(&s_full[w], j & 1);
       tc_fence_after();
-      if (j == ntiles - 1 && L - j * BN < BN) {
-        // Zero V rows past the sequence end before the last PV product.  S_j
-        // complete implies PV_{j-2} complete, hence this V stage's previous
-        // use has landed and the parity below names the current phase (a
-        // wait on an older phase could alias the next, never-completing one).
-        if (alive) alive = mbar_wait(&v_full[st], (j >> 1) & 1);
-        const int first = L - j * BN;
-        uint8_t* sv = smem + Sh::V_OFF + st * Sh::TILE;
+      const int kbase = j * BN;
+      if (w == 0 && j == ntiles - 1 && L - kbase < BN) {
+        // Zero V rows past the sequence end before PV0/PV1 of the last tile.
+        // S0_j complete implies every earlier use of V_j's stage landed, so
+        // this parity names the current phase.
+        const int it_v = 2 * j + 1, st_v = it_v % NS;
+        if (alive) alive = mbar_wait(&ring_full[st_v], (it_v / NS) & 1);
+        const int first = L - kbase;
+        uint8_t* vs = smem + Sh::RING_OFF + st_v * Sh::TILE;
         for (int idx = r; idx < (BN - first) * 16; idx += 128) {
-          const int row = first + idx / 16, ch = idx % 16;
-          *reinterpret_cast<uint4*>(sv + (ch >> 3) * Sh::HALF + row * 128 + (ch & 7) * 16) =
+          const int vr = first + idx / 16, ch = idx % 16;
+          *reinterpret_cast<uint4*>(vs + (ch >> 3) * Sh::HALF + vr * 128 + (ch & 7) * 16) =
               make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
-      float sv[BN];
-#pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t rr[32];
-        tmem_ld32(t_s[st] + lane_off + cc * 32, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[cc * 32 + e] = __uint_as_float(rr[e]);
-      }
-      const int kbase = j * BN;
+      uint32_t sv[BN];
+      tmem_ld32_at<0>(t_s, sv);
+      tmem_ld32_at<32>(t_s + 32, sv);
+      tmem_ld32_at<64>(t_s + 64, sv);
+      tmem_ld32_at<96>(t_s + 96, sv);
+      tmem_wait_ld();
+      const bool masked = kbase + BN - 1 > limit;
       float mx = -INFINITY;
+      if (masked) {
 #pragma unroll
-      for (int e = 0; e < BN; ++e) {
-        const float x = (kbase + e <= limit) ? sv[e] * p.scale_log2 : -INFINITY;
-        sv[e] = x;
-        mx = fmaxf(mx, x);
+        for (int e = 0; e < BN; ++e) {
+          const float x = kbase + e <= limit ? __uint_as_float(sv[e]) : -INFINITY;
+          sv[e] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < BN; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
       }
-      if (mx > m_run + 8.0f) {
-        // raise the running max; rescale l and O (O only exists after tile 0)
-        const float alpha = exp2f(m_run - mx);
+      const float m_tile = mx * sc;  // scale > 0, so the max commutes with it
+      if (m_tile > m_run + 8.0f) {
+        // raise the running max; rescale l and O (O exists after tile 0, and
+        // S_w(j) complete implies PV_w(j-1) complete)
+        const float alpha = exp2f(m_run - m_tile);
         l_run *= alpha;
         if (j > 0) {
-          if (alive) alive = mbar_wait(o_done, (j - 1) & 1);
-          tc_fence_after();
-#pragma unroll
+          // 32 columns at a time: the S row stays live in registers meanwhile
+#pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t rr[32];
-            tmem_ld32(t_o + lane_off + cc * 32, rr);
+            uint32_t ov[32];
+            tmem_ld32(t_o + cc * 32, ov);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st32(t_o + lane_off + cc * 32, rr);
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(t_o + cc * 32, ov);
           }
         }
-        m_run = mx;
+        m_run = m_tile;
       }
-      float rs = 0.f;
+      const float neg_m = -m_run;
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float a = exp2f(sv[cc * 32 + 2 * e] - m_run);
-          const float b = exp2f(sv[cc * 32 + 2 * e + 1] - m_run);
-          rs += a + b;
+          const float a = exp2f(fmaf(__uint_as_float(sv[cc * 32 + 2 * e]), sc, neg_m));
+          const float b = exp2f(fmaf(__uint_as_float(sv[cc * 32 + 2 * e + 1]), sc, neg_m));
+          rs0 += a;
+          rs1 += b;
           pk[e] = MmaOp<T>::pack(a, b);
         }
-        tmem_st16(t_s[st] + lane_off + cc * 16, pk);
+        tmem_st16(t_s + cc * 16, pk);
       }
-      l_run += rs;
+      l_run += rs0 + rs1;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[st]);
+      mbar_arrive(&p_full[w]);
     }
-    // epilogue: O / l for the valid rows, once the last PV product is done
-    // (a one-shot barrier, so the wait cannot alias another phase).
-    if (alive) alive = mbar_wait(o_final, 0);
+    // epilogue: O / l for the valid rows (one-shot barrier per Q tile)
+    if (alive) alive = mbar_wait(&o_final[w], 0);
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + i0 + r) * p.num_q_heads + h) * D;
+    T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + h) * D;
+    uint32_t ov[D];
+    tmem_ld32_at<0>(t_o, ov);
+    tmem_ld32_at<32>(t_o + 32, ov);
+    tmem_ld32_at<64>(t_o + 64, ov);
+    tmem_ld32_at<96>(t_o + 96, ov);
+    tmem_wait_ld();
+    if (row < n) {
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t rr[32];
-      tmem_ld32(t_o + lane_off + cc * 32, rr);
-      tmem_wait_ld();
-      if (r < rows) {
-        uint32_t pk[16];
+      for (int v = 0; v < D / 8; ++v) {
+        uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = MmaOp<T>::pack(__uint_as_float(rr[2 * e]) * inv,
-                                 __uint_as_float(rr[2 * e + 1]) * inv);
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          reinterpret_cast<uint4*>(orow + cc * 32)[v] =
-              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int e = 0; e < 4; ++e)
+          pk[e] = MmaOp<T>::pack(__uint_as_float(ov[8 * v + 2 * e]) * inv,
+                                 __uint_as_float(ov[8 * v + 2 * e + 1]) * inv);
+        reinterpret_cast<uint4*>(orow)[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
   }
