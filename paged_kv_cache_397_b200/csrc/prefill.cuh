@@ -287,20 +287,21 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
       tmem_ld32_at<64>(t_s + 64, sv);
       tmem_ld32_at<96>(t_s + 96, sv);
       tmem_wait_ld();
-      const bool masked = kbase + BN - 1 > limit;
-      float mx = -INFINITY;
-      if (masked) {
+      if (kbase + BN - 1 > limit) {  // only tiles that reach past this row's limit
 #pragma unroll
-        for (int e = 0; e < BN; ++e) {
-          const float x = kbase + e <= limit ? __uint_as_float(sv[e]) : -INFINITY;
-          sv[e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < BN; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
+        for (int e = 0; e < BN; ++e)
+          if (kbase + e > limit) sv[e] = __float_as_uint(-INFINITY);
       }
-      const float m_tile = mx * sc;  // scale > 0, so the max commutes with it
+      // row max: four independent chains of three-input max
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < BN; e += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(sv[e + 4]), __uint_as_float(sv[e + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(sv[e + 6]), __uint_as_float(sv[e + 7]));
+      }
+      const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc;  // scale > 0 commutes
       if (m_tile > m_run + 8.0f) {
         // raise the running max; rescale l and O (O exists after tile 0, and
         // S_w(j) complete implies PV_w(j-1) complete)
@@ -320,22 +321,29 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
         }
         m_run = m_tile;
       }
-      const float neg_m = -m_run;
-      float rs0 = 0.f, rs1 = 0.f;
+      // P = 2^(S * scale - m): packed FMA, SFU exp2, packed row sums
+      const uint64_t sc2 = f2_pack(sc, sc), negm2 = f2_pack(-m_run, -m_run);
+      uint64_t rsum[4] = {0, 0, 0, 0};  // four packed partial sums
 #pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t pk[16];
+      for (int cc = 0; cc < BN / 16; ++cc) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = exp2f(fmaf(__uint_as_float(sv[cc * 32 + 2 * e]), sc, neg_m));
-          const float b = exp2f(fmaf(__uint_as_float(sv[cc * 32 + 2 * e + 1]), sc, neg_m));
-          rs0 += a;
-          rs1 += b;
+        for (int e = 0; e < 8; ++e) {
+          const int x = cc * 16 + 2 * e;
+          float a, b;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), sc2,
+                           negm2),
+                    a, b);
+          a = ex2_approx(a);
+          b = ex2_approx(b);
+          rsum[e & 3] = f2_add(rsum[e & 3], f2_pack(a, b));
           pk[e] = MmaOp<T>::pack(a, b);
         }
-        tmem_st16(t_s + cc * 16, pk);
+        tmem_st8(t_s + cc * 8, pk);
       }
-      l_run += rs0 + rs1;
+      float l0, l1;
+      f2_unpack(f2_add(f2_add(rsum[0], rsum[1]), f2_add(rsum[2], rsum[3])), l0, l1);
+      l_run += l0 + l1;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
