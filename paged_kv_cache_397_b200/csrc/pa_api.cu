@@ -151,6 +151,12 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   auto kern = pa::prefill_kernel<T, BS>;
   static bool configured = false;
   if (!configured) {
+    // The kernel's setmaxnreg split assumes at least MIN_LAUNCH_REGS registers
+    // per thread at launch; with fewer, its register increase could never be
+    // granted, so such a build is refused rather than launched.
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return PA_ERR_CUDA;
+    if (attr.numRegs < Sh::MIN_LAUNCH_REGS) return PA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Sh::SMEM_BYTES) != cudaSuccess)
       return PA_ERR_CUDA;

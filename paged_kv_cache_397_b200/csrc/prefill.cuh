@@ -56,8 +56,16 @@ struct PrefillShape {
   static constexpr int BM = 128;                // rows per Q tile
   static constexpr int NQ = 2;                  // Q tiles per CTA
   static constexpr int BN = 128;                // keys per K/V tile
-  static constexpr int THREADS = 10 * 32;
-  static constexpr int TMA_WARP = 8, MMA_WARP = 9;
+  static constexpr int THREADS = 12 * 32;       // 3 warpgroups
+  static constexpr int TMA_WARP = 8, MMA_WARP = 9;  // warps 10-11 idle
+  // Registers per thread after setmaxnreg: softmax warpgroups grow, the
+  // producer warpgroup shrinks.  2*128*200 + 128*96 = 63488 must not exceed
+  // the launch allocation THREADS * MIN_LAUNCH_REGS = 64512, so the host
+  // refuses to launch a build whose kernel has fewer than MIN_LAUNCH_REGS.
+  static constexpr uint32_t SOFTMAX_REGS = 200, PRODUCER_REGS = 96;
+  static constexpr int MIN_LAUNCH_REGS = 168;
+  static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= THREADS * MIN_LAUNCH_REGS,
+                "register split exceeds the launch allocation");
   static constexpr int HALF = 128 * 128;        // 128 rows x 64 columns x 2 bytes
   static constexpr int TILE = 2 * HALF;         // 128 x 128 x 2 bytes = 32 KB
   static constexpr int NSTAGE = 4;              // K/V ring stages (K_j, V_j alternate)
@@ -155,6 +163,9 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+    // producer warpgroup: TMA warp, MMA warp, two idle warps
+    setmaxnreg_dec<Sh::PRODUCER_REGS>();
   if (warp == Sh::TMA_WARP) {
     // ------------------------------------------------------------ TMA warp
     const uint64_t pol_kv = l2_policy_evict_last();
@@ -250,8 +261,10 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
         }
       }
     }
+  }
   } else {
     // -------------------------------------------------- softmax warpgroups
+    setmaxnreg_inc<Sh::SOFTMAX_REGS>();
     const int w = warp >> 2;                       // Q tile of this warpgroup
     const int r = threadIdx.x & 127;               // row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
