@@ -33,7 +33,7 @@ __all__ = [
     "PagedDecodeInputs", "PrefillChunkInputs", "WORKLOADS", "make_workload",
     "tiny_decode", "llama2_13b_decode", "llama3_8b_gqa_decode",
     "shared_prefix_cow", "long_context_decode", "chunked_prefill", "random_decode",
-    "NAN_FILL",
+    "llama3_8b_gqa_decode_fp8", "NAN_FILL", "FP8_NAN_CODE",
 ]
 
 NAN_FILL = float("nan")
@@ -68,6 +68,9 @@ class PagedDecodeInputs:
     new_value: Optional[torch.Tensor]
     free_blocks: torch.Tensor
     scale: float
+    # FP8 caches only: the per-cache scale (codes stand for value * scale);
+    # None for fp16 / bf16 caches
+    kv_scale: Optional[float] = None
     # copy-on-write workload only: the shared physical blocks and, per
     # sequence, a fresh destination block for the diverging block
     shared_blocks: Optional[torch.Tensor] = None
@@ -139,15 +142,40 @@ def _randn(gen: torch.Generator, shape, dtype: torch.dtype, chunk: int = 1 << 24
     return out
 
 
-def _pool(gen, num_blocks, num_kv_heads, block_size, head_dim, dtype, used_blocks):
-    kc = _randn(gen, (num_blocks, num_kv_heads, block_size, head_dim), dtype)
-    vc = _randn(gen, (num_blocks, num_kv_heads, block_size, head_dim), dtype)
+def _pool(gen, num_blocks, num_kv_heads, block_size, head_dim, dtype, used_blocks,
+          fp8_scale=None):
+    shape = (num_blocks, num_kv_heads, block_size, head_dim)
+    if fp8_scale is None:
+        kc = _randn(gen, shape, dtype)
+        vc = _randn(gen, shape, dtype)
+    else:
+        # FP8 E4M3 codes of N(0,1) / scale, drawn through torch's float8 cast
+        kc = _fp8_codes(gen, shape, fp8_scale)
+        vc = _fp8_codes(gen, shape, fp8_scale)
     used = torch.zeros(num_blocks, dtype=torch.bool)
     used[used_blocks] = True
     free = torch.nonzero(~used).flatten()
-    kc[free] = NAN_FILL
-    vc[free] = NAN_FILL
+    if fp8_scale is None:
+        kc[free] = NAN_FILL
+        vc[free] = NAN_FILL
+    else:
+        kc[free] = FP8_NAN_CODE
+        vc[free] = FP8_NAN_CODE
     return kc, vc, free
+
+
+FP8_NAN_CODE = 0x7F
+
+
+def _fp8_codes(gen, shape, scale, chunk: int = 1 << 24) -> torch.Tensor:
+    out = torch.empty(shape, dtype=torch.uint8)
+    flat = out.view(-1)
+    n = flat.numel()
+    for i in range(0, n, chunk):
+        j = min(n, i + chunk)
+        x = torch.randn(j - i, generator=gen, dtype=torch.float32) / scale
+        flat[i:j] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out
 
 
 def _tables_from_counts(perm: torch.Tensor, counts, max_blocks: int, start: int = 0):
@@ -161,14 +189,14 @@ def _tables_from_counts(perm: torch.Tensor, counts, max_blocks: int, start: int 
 
 
 def _decode_batch(name, seed, gen, lens, *, dtype, block_size, hq, hkv, d, append,
-                  pool_factor=1.25, pool_blocks=None):
+                  pool_factor=1.25, pool_blocks=None, fp8_scale=None):
     lens = [int(x) for x in lens]
     counts = [_ceil_div(L + (1 if append else 0), block_size) for L in lens]
     need = sum(counts)
     num_blocks = pool_blocks if pool_blocks is not None else int(math.ceil(pool_factor * need))
     perm = torch.randperm(num_blocks, generator=gen)
-    bt, used = _tables_from_counts(perm, counts, max(counts))
-    kc, vc, free = _pool(gen, num_blocks, hkv, block_size, d, dtype, perm[:used])
+    bt, used = _tables_from_counts(perm, counts, max(1, max(counts)))
+    kc, vc, free = _pool(gen, num_blocks, hkv, block_size, d, dtype, perm[:used], fp8_scale)
     q = _randn(gen, (len(lens), hq, d), dtype)
     nk = _randn(gen, (len(lens), hkv, d), dtype) if append else None
     nv = _randn(gen, (len(lens), hkv, d), dtype) if append else None
@@ -177,7 +205,7 @@ def _decode_batch(name, seed, gen, lens, *, dtype, block_size, hq, hkv, d, appen
         num_kv_heads=hkv, head_dim=d, num_blocks=num_blocks,
         context_lens=torch.tensor(lens, dtype=torch.int32), block_tables=bt,
         key_cache=kc, value_cache=vc, query=q, new_key=nk, new_value=nv,
-        free_blocks=free, scale=1.0 / math.sqrt(d))
+        free_blocks=free, scale=1.0 / math.sqrt(d), kv_scale=fp8_scale)
 
 
 def tiny_decode(seed: int = 0) -> PagedDecodeInputs:
@@ -280,19 +308,33 @@ def chunked_prefill(seed: int = 4, block_size: int = 16, num_seqs: int = 8, ctx:
         new_value=nv, free_blocks=free, scale=1.0 / math.sqrt(d))
 
 
+def llama3_8b_gqa_decode_fp8(seed: int = 2, num_seqs: int = 256,
+                             block_size: int = 16) -> PagedDecodeInputs:
+    """The Llama-3-8B-shaped GQA decode batch with an FP8 (E4M3) K/V pool:
+    same lengths and block shuffle as llama3_8b_gqa_decode; the pool holds
+    codes of N(0,1) / (1/32), i.e. values N(0,1) under a scale of 1/32; the
+    query and the appended token stay bf16."""
+    gen = torch.Generator().manual_seed(seed)
+    lens = torch.randint(128, 4096 + 1, (num_seqs,), generator=gen).tolist()
+    return _decode_batch(f"llama3_8b_gqa_decode_fp8_{num_seqs}seq_L128-4096_h32kv8_d128_e4m3_B{block_size}",
+                         seed, gen, lens, dtype=torch.bfloat16, block_size=block_size,
+                         hq=32, hkv=8, d=128, append=True, fp8_scale=1.0 / 32)
+
+
 def random_decode(seed: int, lens, *, dtype=torch.float16, block_size=16, hq=4, hkv=4, d=64,
-                  append=True, pool_factor=1.5) -> PagedDecodeInputs:
+                  append=True, pool_factor=1.5, fp8_scale=None) -> PagedDecodeInputs:
     """A small decode batch with caller-chosen lengths (for edge cases and sweeps)."""
     gen = torch.Generator().manual_seed(seed)
     return _decode_batch(f"random_decode_s{seed}", seed, gen, lens, dtype=dtype,
                          block_size=block_size, hq=hq, hkv=hkv, d=d, append=append,
-                         pool_factor=pool_factor)
+                         pool_factor=pool_factor, fp8_scale=fp8_scale)
 
 
 WORKLOADS = {
     "tiny_decode": tiny_decode,
     "llama2_13b_decode": llama2_13b_decode,
     "llama3_8b_gqa_decode": llama3_8b_gqa_decode,
+    "llama3_8b_gqa_decode_fp8": llama3_8b_gqa_decode_fp8,
     "shared_prefix_cow": shared_prefix_cow,
     "long_context_decode": long_context_decode,
     "chunked_prefill": chunked_prefill,
