@@ -54,7 +54,9 @@ typedef enum {
   PA_ERR_CUDA = 5
 } pa_status;
 
-typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+/* Element types.  PA_FP8_E4M3 is a cache-only type (1 byte per element; see
+ * pa_reshape_and_cache_fp8 / pa_decode_fp8); pa_copy_blocks accepts all three. */
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 /* Bits of the device error word (pa_get_device_error). */
 #define PA_DEVERR_SLOT_RANGE 0x1u    /* slot_mapping entry >= num_blocks * block_size   */
@@ -119,12 +121,34 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *key_cac
  * value_cache[dst] = value_cache[src] (all heads, slots and dims; bit copy).
  * dst ids must be distinct and no dst may also be a src.
  *   key_cache, value_cache  in/out  T[num_blocks][num_kv_heads][block_size][head_dim]
+ *                                   (T = dtype; PA_FP8_E4M3 caches are 1 byte per element)
  *   block_pairs             in      int64[num_pairs][2] = {src, dst}
  * A pair with an id outside [0, num_blocks) is skipped and sets PA_DEVERR_BLOCK_RANGE.
  */
 pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *block_pairs,
                          int num_pairs, int num_kv_heads, int head_dim, int block_size,
                          int num_blocks, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_reshape_and_cache_fp8 — pa_reshape_and_cache into FP8 (E4M3) caches.
+ *   "PagedAttention: KV cache as virtual memory", "Deep dive" and
+ *   "Interviewer follow-ups" (an FP8 KV cache halves the bytes per block and
+ *   raises the number of sequences that fit).  The pages fix no encoding or
+ *   scaling; this library's reading: OCP E4M3 without infinities (bias 7,
+ *   max 448), one fp32 scale per cache, a code standing for value * scale.
+ * code = nearest E4M3 of (fp32(x) / scale) — IEEE fp32 division, ties to the
+ * even code, magnitudes above 448 saturate to 448.  Slot -1 skips a token.
+ *   key, value              in      T[num_tokens][num_kv_heads][head_dim], T = dtype
+ *   key_cache, value_cache  in/out  uint8[num_blocks][num_kv_heads][block_size][head_dim]
+ *   slot_mapping            in      int64[num_tokens]
+ *   k_scale, v_scale        positive finite fp32 scales of the two caches
+ * head_dim must be a multiple of 16.  Out-of-range slots: as pa_reshape_and_cache.
+ */
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, uint8_t *key_cache,
+                                   uint8_t *value_cache, const int64_t *slot_mapping,
+                                   int num_tokens, int num_kv_heads, int head_dim,
+                                   int block_size, int num_blocks, float k_scale, float v_scale,
+                                   pa_dtype dtype, pa_stream_t stream);
 
 /*
  * pa_decode_partition_tokens — the split-KV partition length pa_decode uses
@@ -175,6 +199,24 @@ pa_status pa_decode(void *out, const void *query, const void *key_cache, const v
                     int num_blocks, int max_blocks_per_seq, int max_seq_len,
                     int partition_tokens, float scale, pa_dtype dtype, void *workspace,
                     size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_decode_fp8 — pa_decode over FP8 (E4M3) caches (see pa_reshape_and_cache_fp8
+ * for the encoding).  Attention is computed over the values code * k_scale and
+ * code * v_scale; the query and output are fp16 or bf16 (`dtype`).  The
+ * products run on fp16 tensor-core MMAs with fp32 accumulation: E4M3 codes
+ * are exact in fp16, the query is rounded to fp16 (exact for |q| in fp16's
+ * normal range).  Same arguments, partitioning, workspace
+ * (pa_decode_workspace_size with the same sizes), determinism and error
+ * behaviour as pa_decode.  head_dim must be 128.
+ */
+pa_status pa_decode_fp8(void *out, const void *query, const uint8_t *key_cache,
+                        const uint8_t *value_cache, const int32_t *block_tables,
+                        const int32_t *seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                        int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                        int max_seq_len, int partition_tokens, float scale, float k_scale,
+                        float v_scale, pa_dtype dtype, void *workspace, size_t workspace_bytes,
+                        pa_stream_t stream);
 
 /*
  * pa_decode_static_workspace — pa_decode for callers that cannot allocate

@@ -27,14 +27,15 @@ __all__ = [
     "pa_decode_workspace_size", "pa_decode", "pa_decode_static_workspace", "pa_prefill_chunk",
     "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
-    "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16",
+    "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
 ]
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = 0, 1, 2, 3
 PA_ERR_OUT_OF_RANGE, PA_ERR_CUDA = 4, 5
-PA_F16, PA_BF16 = 0, 1
+PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 PA_DEVERR_SLOT_RANGE, PA_DEVERR_BLOCK_RANGE = 0x1, 0x2
 PA_DEVERR_SEQ_RANGE, PA_DEVERR_WAIT_TIMEOUT = 0x4, 0x8
 
@@ -54,6 +55,9 @@ _SIGS = {
                        _p, _sz, _p]),
     "pa_decode_static_workspace": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                                         _i, _i, _f, _i, _p]),
+    "pa_reshape_and_cache_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _i, _p]),
+    "pa_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _f,
+                           _f, _i, _p, _sz, _p]),
     "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                               _i, _f, _i, _p]),
     "pa_get_device_error": (_i, [ctypes.POINTER(ctypes.c_uint), _p]),
@@ -93,12 +97,15 @@ def _check(fn: str, status: int) -> None:
         raise PAError(fn, status)
 
 
-def _dtype_code(t: torch.Tensor) -> int:
+def _dtype_code(t: torch.Tensor, allow_fp8: bool = False) -> int:
     if t.dtype == torch.float16:
         return PA_F16
     if t.dtype == torch.bfloat16:
         return PA_BF16
-    raise ValueError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+    if allow_fp8 and t.dtype == torch.uint8:
+        return PA_FP8_E4M3
+    raise ValueError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16"
+                     + (" or uint8 (E4M3 codes)" if allow_fp8 else ""))
 
 
 def _ptr(t, name: str, dtype=None, ndim=None) -> Optional[int]:
@@ -177,7 +184,53 @@ def pa_copy_blocks(key_cache, value_cache, block_pairs, stream=None):
     _check("pa_copy_blocks", lib().pa_copy_blocks(
         _ptr(key_cache, "key_cache"), _ptr(value_cache, "value_cache"),
         _ptr(block_pairs, "block_pairs", torch.int64, 2), int(block_pairs.shape[0]), hkv, d, bs,
-        nb, _dtype_code(key_cache), _stream(stream)))
+        nb, _dtype_code(key_cache, allow_fp8=True), _stream(stream)))
+
+
+def pa_reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale,
+                             v_scale, stream=None):
+    """Scatter new fp16/bf16 K/V rows into FP8 (E4M3, uint8) caches (include/pa.h)."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if key_cache.dtype != torch.uint8:
+        raise ValueError("FP8 caches are uint8 tensors of E4M3 codes")
+    if key.shape != value.shape or key.dim() != 3 or tuple(key.shape[1:]) != (hkv, d):
+        raise ValueError("key/value must be [num_tokens][num_kv_heads][head_dim] like the cache")
+    if key.dtype != value.dtype:
+        raise ValueError("key and value dtypes differ")
+    if slot_mapping.numel() != key.shape[0]:
+        raise ValueError("slot_mapping needs one entry per token")
+    _check("pa_reshape_and_cache_fp8", lib().pa_reshape_and_cache_fp8(
+        _ptr(key, "key"), _ptr(value, "value"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(slot_mapping, "slot_mapping", torch.int64, 1),
+        int(key.shape[0]), hkv, d, bs, nb, float(k_scale), float(v_scale), _dtype_code(key),
+        _stream(stream)))
+
+
+def pa_decode_fp8(out, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len,
+                  scale, k_scale, v_scale, workspace=None, partition_tokens=0, stream=None):
+    """Paged decode over FP8 (E4M3, uint8) caches; fp16/bf16 query and output."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if key_cache.dtype != torch.uint8:
+        raise ValueError("FP8 caches are uint8 tensors of E4M3 codes")
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs][num_q_heads][head_dim]")
+    if out.dtype != query.dtype:
+        raise ValueError("out dtype must match the query")
+    S, hq = int(query.shape[0]), int(query.shape[1])
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.numel() != S:
+        raise ValueError("block_tables / seq_lens do not match the batch")
+    need = pa_decode_workspace_size(S, hq, hkv, d, bs, max_seq_len, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_fp8", lib().pa_decode_fp8(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(seq_lens, "seq_lens", torch.int32, 1), S, hq, hkv, d, bs, nb,
+        int(block_tables.shape[1]), int(max_seq_len), int(partition_tokens), float(scale),
+        float(k_scale), float(v_scale), _dtype_code(query), ws_ptr, ws_bytes, _stream(stream)))
+    return out
 
 
 def pa_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len) -> int:

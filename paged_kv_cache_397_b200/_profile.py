@@ -1,6 +1,7 @@
 """Small, self-contained cases of the hot kernels for ncu captures.
 
     python -m paged_kv_cache_397_b200._profile decode  --seqs 32
+    python -m paged_kv_cache_397_b200._profile decode-fp8 --seqs 64
     python -m paged_kv_cache_397_b200._profile prefill --seqs 4 [--block-size 16]
 
 Each case builds a scaled-down copy of a bench workload (same shapes, head
@@ -41,6 +42,21 @@ def decode_case(seqs: int, reps: int = 3):
     print(f"decode case: {w.name}, K/V bytes per launch {kv}")
 
 
+def decode_fp8_case(seqs: int, reps: int = 3):
+    w = synth.llama3_8b_gqa_decode_fp8(num_seqs=seqs)
+    d = torch.device("cuda:0")
+    kc, vc, bt = w.key_cache.to(d), w.value_cache.to(d), w.block_tables.to(d)
+    lens = (w.context_lens + 1).to(d)
+    q = w.query.to(d)
+    out = torch.empty_like(q)
+    max_len = int(lens.max())
+    for _ in range(reps):
+        pa.pa_decode_fp8(out, q, kc, vc, bt, lens, max_len, w.scale, w.kv_scale, w.kv_scale)
+    torch.cuda.synchronize()
+    kv = 2 * w.num_kv_heads * w.head_dim * int(lens.sum())
+    print(f"decode-fp8 case: {w.name}, K/V bytes per launch {kv}")
+
+
 def prefill_case(seqs: int, block_size: int, reps: int = 3):
     p = synth.chunked_prefill(num_seqs=seqs, block_size=block_size)
     d = torch.device("cuda:0")
@@ -59,13 +75,15 @@ def prefill_case(seqs: int, block_size: int, reps: int = 3):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode", "prefill"])
+    ap.add_argument("case", choices=["decode", "decode-fp8", "prefill"])
     ap.add_argument("--seqs", type=int, default=None)
     ap.add_argument("--block-size", type=int, default=16)
     a = ap.parse_args()
     pa.lib()
     if a.case == "decode":
         decode_case(a.seqs or 32)
+    elif a.case == "decode-fp8":
+        decode_fp8_case(a.seqs or 64)
     else:
         prefill_case(a.seqs or 4, a.block_size)
     if pa.pa_get_device_error():

@@ -5,6 +5,8 @@
 // launch latency and one HBM round trip, not by bandwidth.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "ptx.cuh"
 
 namespace pa {
@@ -72,6 +74,60 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
   const uint4 vv = __ldg(value + src);
   key_cache[dst] = kv;
   value_cache[dst] = vv;
+}
+
+// FP8 (E4M3) cache write: one thread per 16 elements of one (token, kv head)
+// row of K and of V.  Each value is divided by its cache's scale in fp32
+// (IEEE division) and rounded to the nearest E4M3 code, ties to even,
+// magnitudes above 448 saturating ("PagedAttention: KV cache as virtual
+// memory", "Interviewer follow-ups": an FP8 KV cache halves the bytes per
+// block; the encoding and the per-cache scale are this library's reading).
+template <typename T>
+__global__ void reshape_and_cache_fp8_kernel(const T* __restrict__ key, const T* __restrict__ value,
+                                             uint8_t* __restrict__ key_cache,
+                                             uint8_t* __restrict__ value_cache,
+                                             const int64_t* __restrict__ slot_mapping,
+                                             int num_tokens, int num_kv_heads, int head_dim,
+                                             int block_size, int64_t num_slots, float k_scale,
+                                             float v_scale) {
+  const int CH = head_dim / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)num_tokens * num_kv_heads * CH;
+  if (idx >= total) return;
+  const int c = (int)(idx % CH);
+  const int64_t th = idx / CH;  // token * Hkv + head
+  const int h = (int)(th % num_kv_heads);
+  const int64_t t = th / num_kv_heads;
+  const int64_t slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (c == 0) record_error(PA_DEVERR_SLOT_RANGE);
+    return;
+  }
+  const int64_t b = slot / block_size, off = slot % block_size;
+  const int64_t src = th * head_dim + c * 16;
+  const int64_t dst = ((b * num_kv_heads + h) * block_size + off) * head_dim + c * 16;
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    const T* in = (kv == 0 ? key : value) + src;
+    const float sc = kv == 0 ? k_scale : v_scale;
+    uint4 raw[2];
+    raw[0] = __ldg(reinterpret_cast<const uint4*>(in));
+    raw[1] = __ldg(reinterpret_cast<const uint4*>(in) + 1);
+    const T* x = reinterpret_cast<const T*>(raw);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+          make_float2(float(x[4 * q]) / sc, float(x[4 * q + 1]) / sc), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(float(x[4 * q + 2]) / sc, float(x[4 * q + 3]) / sc), __NV_SATFINITE,
+          __NV_E4M3);
+      w[q] = (lo & 0xFFFF) | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>((kv == 0 ? key_cache : value_cache) + dst) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 // One CTA per (pair, K-or-V); each thread moves kPerThread 16-byte chunks,

@@ -14,23 +14,35 @@
 //    and applies it to all G query heads of the group.
 //  * One producer warp streams the (block, KV head) tiles — each a
 //    contiguous block_size x head_dim run of the pool — into a ring of shared
-//    memory stages with TMA (cp.async.bulk.tensor, 128-byte swizzle, one
-//    16-byte-aligned box per 64 columns), completing on mbarriers.  The
+//    memory stages with TMA (cp.async.bulk.tensor, 128-byte swizzle, boxes
+//    starting on 16-byte boundaries), completing on mbarriers.  The
 //    block-table entries of a partition are fetched once, coalesced, by the
 //    producer warp.
 //  * Four consumer warps take blocks round-robin.  Each 16-token sub-tile is
 //    a tiny GEMM pair on the warp-level tensor-core path (mma.sync m16n8k16,
 //    fp32 accumulate): S^T = K Q^T puts tokens on M and the (padded) query
 //    heads on N; P^T is moved into the B-operand layout in registers with
-//    movmatrix; O^T += V^T P^T reads V transposed with ldmatrix.trans.  Online
-//    softmax (running max, exp2, rescale) stays in registers; the max uses
-//    warp shuffles.  Decode is HBM-bound, so the point of the tensor path is
-//    only to keep ALU issue far below the memory time.
+//    movmatrix; O^T += V^T P^T.  Online softmax (running max, exp2, rescale)
+//    stays in registers; the max uses warp shuffles.  Decode is HBM-bound, so
+//    the point of the tensor path is only to keep ALU issue far below the
+//    memory time.
 //  * Warps merge their softmax states in shared memory in a fixed order.  A
 //    sequence with one partition writes the final row; otherwise the
 //    partition writes (m, l, acc) to the workspace and decode_reduce_kernel
 //    combines partitions with the log-sum-exp rule in partition order.
+//
+// Two cache formats share that skeleton through a tile policy:
+//  * HalfTiles — fp16 / bf16 caches; K and V^T fragments come from the
+//    swizzled tiles through ldmatrix / ldmatrix.trans; MMA in the cache type.
+//  * E4m3Tiles — FP8 (E4M3) caches with one scale per cache ("PagedAttention:
+//    KV cache as virtual memory", "Interviewer follow-ups": FP8 KV halves the
+//    bytes per block).  Fragments are built from 16-byte / 4-byte shared loads
+//    and converted e4m3x2 -> f16x2; MMA in fp16 (the query is rounded to fp16;
+//    E4M3 values are exact in fp16).  k_scale is folded into the softmax scale
+//    and v_scale multiplies the output once.
 #pragma once
+
+#include <cuda_fp8.h>
 
 #include "ptx.cuh"
 
@@ -47,33 +59,292 @@ struct DecodeParams {
   int num_blocks, max_blocks_per_seq;
   int part_blocks;           // logical blocks per partition
   int max_parts;             // gridDim.x
-  float scale_log2;          // softmax scale * log2(e)
+  float scale_log2;          // softmax scale * log2(e) (FP8: also * k_scale)
+  float v_scale;             // FP8: multiplies the output; 1 otherwise
 };
 
-template <typename T, int D, int BS, int NT>
+// ------------------------------------------------------------------ tiles
+// Address of byte `col` of row `row` in a tile of 128-byte rows written by a
+// TMA box with 128-byte swizzle (16-byte chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t sw128(uint32_t base, int row, int col) {
+  return base + row * 128 + ((((col >> 4) ^ (row & 7)) << 4) | (col & 15));
+}
+
+// fp16 / bf16 cache: a (block, kv head) tile is BS rows x D columns, stored as
+// D/64 column groups of BS x 128 bytes.
+template <typename T, int D_, int BS>
+struct HalfTiles {
+  using Elem = T;   // query / output type
+  using MmaT = T;   // MMA operand type
+  static constexpr int D = D_;
+  static constexpr int BOXES = D / 64;              // TMA boxes per tile
+  static constexpr int BOX_BYTES = BS * 128;
+  static constexpr int TILE_BYTES = BS * D * 2;
+  static constexpr int NS = BS == 16 ? 8 : 4;        // ring depth
+  static constexpr int ZERO_CHUNKS_PER_ROW = BOXES * 8;
+
+  __device__ static void issue(uint8_t* sk, uint8_t* sv, const CUtensorMap* mk,
+                               const CUtensorMap* mv, int row, uint64_t* bar, uint64_t pol) {
+#pragma unroll
+    for (int h = 0; h < BOXES; ++h) {
+      tma_load_2d(sk + h * BOX_BYTES, mk, h * 64, row, bar, pol);
+      tma_load_2d(sv + h * BOX_BYTES, mv, h * 64, row, bar, pol);
+    }
+  }
+  // 16-byte chunk `idx` of V row `r` (for zeroing rows past the sequence end)
+  __device__ static uint8_t* zero_chunk(uint8_t* v, int r, int idx) {
+    return v + (idx >> 3) * BOX_BYTES + r * 128 + (idx & 7) * 16;
+  }
+  // Q^T as the B operand: k = head dim in natural order
+  template <int NT>
+  __device__ static void load_q(uint32_t (&qf)[D / 16][NT][2], const T* qbase, int G,
+                                int lane) {
+    const int c4 = lane & 3, r4 = lane >> 2;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 8 + r4;
+#pragma unroll
+      for (int kt = 0; kt < D / 16; ++kt) {
+        uint32_t b0 = 0, b1 = 0;
+        if (g < G) {
+          const uint32_t* row = reinterpret_cast<const uint32_t*>(qbase + (size_t)g * D);
+          b0 = __ldg(row + (kt * 16 + 2 * c4) / 2);
+          b1 = __ldg(row + (kt * 16 + 2 * c4 + 8) / 2);
+        }
+        qf[kt][nt][0] = b0;
+        qf[kt][nt][1] = b1;
+      }
+    }
+  }
+  // S^T (16 tokens of sub-tile mt x 8*NT heads) = K Q^T
+  template <int NT>
+  __device__ static void qk(float (&sacc)[NT][4], const uint8_t* tile, int mt,
+                            const uint32_t (&qf)[D / 16][NT][2], int lane) {
+    qk_at<NT>(sacc, smem_u32(tile), mt, qf, lane);
+  }
+  template <int NT>
+  __device__ static void qk_at(float (&sacc)[NT][4], uint32_t sk, int mt,
+                            const uint32_t (&qf)[D / 16][NT][2], int lane) {
+    float acc2[NT][4];  // odd k-steps accumulate separately (two shorter MMA chains)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc2[nt][e] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < D / 16; ++kt) {
+      const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int chunk = (kt & 3) * 2 + (lane >> 4);
+      const uint32_t addr = sk + (kt >> 2) * BOX_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4);
+      uint32_t a[4];
+      ldmatrix_x4(a, addr);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        MmaOp<MmaT>::run((kt & 1) ? acc2[nt] : sacc[nt], a, qf[kt][nt][0], qf[kt][nt][1]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] += acc2[nt][e];
+  }
+  // O^T (D x 8*NT) += V^T P^T for sub-tile mt
+  template <int NT>
+  __device__ static void pv(float (&o)[D / 16][NT][4], const uint8_t* tile, int mt,
+                            const uint32_t (&pb)[NT][2], int lane) {
+    pv_at<NT>(o, smem_u32(tile), mt, pb, lane);
+  }
+  template <int NT>
+  __device__ static void pv_at(float (&o)[D / 16][NT][4], uint32_t sv, int mt,
+                            const uint32_t (&pb)[NT][2], int lane) {
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      const int j = lane >> 3;
+      const int trow = mt * 16 + (lane & 7) + (j >> 1) * 8;
+      const int dcol = dt * 16 + (j & 1) * 8;
+      const int chunk = (dcol & 63) >> 3;
+      const uint32_t addr =
+          sv + (dcol >> 6) * BOX_BYTES + trow * 128 + ((chunk ^ (trow & 7)) << 4);
+      uint32_t a[4];
+      ldmatrix_x4_trans(a, addr);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) MmaOp<MmaT>::run(o[dt][nt], a, pb[nt][0], pb[nt][1]);
+    }
+  }
+  // head-dim index of accumulator element o[dt][.][e] of lane row r4
+  __device__ static int out_d(int dt, int e, int r4) { return dt * 16 + r4 + (e >> 1) * 8; }
+};
+
+// FP8 E4M3 cache, head_dim 128: a tile is BS rows x 128 bytes (one TMA box).
+// Q K^T contracts over the head dim in the permuted order d = 32c + 4kt + j
+// (c = lane % 4, kt = k-step, j = 0..3), so lane c reads bytes [32c, 32c+32)
+// of a K row with two 16-byte loads.  O^T keeps head-dim rows in the permuted
+// order d = 32p + 4r + b (p = m-tile pair, r = lane / 4, b = byte), so the
+// V^T fragments come from one 4-byte word per token row; byte_perm pairs two
+// token rows along the contraction (token) axis.
+template <typename T, int BS>
+struct E4m3Tiles {
+  using Elem = T;
+  using MmaT = __half;
+  static constexpr int D = 128;
+  static constexpr int BOXES = 1;
+  static constexpr int BOX_BYTES = BS * 128;
+  static constexpr int TILE_BYTES = BS * 128;
+  static constexpr int NS = BS == 16 ? 16 : 8;
+  static constexpr int ZERO_CHUNKS_PER_ROW = 8;
+
+  __device__ static void issue(uint8_t* sk, uint8_t* sv, const CUtensorMap* mk,
+                               const CUtensorMap* mv, int row, uint64_t* bar, uint64_t pol) {
+    tma_load_2d(sk, mk, 0, row, bar, pol);
+    tma_load_2d(sv, mv, 0, row, bar, pol);
+  }
+  __device__ static uint8_t* zero_chunk(uint8_t* v, int r, int idx) {
+    return v + r * 128 + idx * 16;
+  }
+  // four E4M3 codes (one 32-bit word) -> two f16x2 words (bytes 0-1, 2-3)
+  __device__ static void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+  }
+  __device__ static uint32_t f16_pair(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+  template <int NT>
+  __device__ static void load_q(uint32_t (&qf)[D / 16][NT][2], const T* qbase, int G,
+                                int lane) {
+    const int c4 = lane & 3, r4 = lane >> 2;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 8 + r4;
+#pragma unroll
+      for (int kt = 0; kt < D / 16; ++kt) {
+        uint32_t b0 = 0, b1 = 0;
+        if (g < G) {
+          const T* row = qbase + (size_t)g * D + 32 * c4 + 4 * kt;
+          b0 = f16_pair(float(row[0]), float(row[1]));
+          b1 = f16_pair(float(row[2]), float(row[3]));
+        }
+        qf[kt][nt][0] = b0;
+        qf[kt][nt][1] = b1;
+      }
+    }
+  }
+  // Shared-memory tile reads are plain loads through the generic pointer of
+  // the tile (ordered after the stage's barrier wait, free to be scheduled
+  // early against register-only work).
+  // Tile reads are volatile shared loads: kept in program order they
+  // measured faster here than compiler-scheduled loads.
+  template <typename V>
+  __device__ static V lds(const uint8_t* tile, int row, int col);
+  template <int NT>
+  __device__ static void qk(float (&sacc)[NT][4], const uint8_t* sk, int mt,
+                            const uint32_t (&qf)[D / 16][NT][2], int lane) {
+    const int c4 = lane & 3, r4 = lane >> 2;
+    const int r_lo = mt * 16 + r4, r_hi = r_lo + 8;
+    uint4 lo[2], hi[2];  // bytes [32c, 32c+32) of rows r_lo, r_hi
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      lo[h] = lds<uint4>(sk, r_lo, 32 * c4 + 16 * h);
+      hi[h] = lds<uint4>(sk, r_hi, 32 * c4 + 16 * h);
+    }
+    float acc2[NT][4];  // odd k-steps accumulate separately (two shorter MMA chains)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc2[nt][e] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < D / 16; ++kt) {
+      const uint4& L = lo[kt >> 2];
+      const uint4& H = hi[kt >> 2];
+      const uint32_t wl = (kt & 3) == 0 ? L.x : (kt & 3) == 1 ? L.y : (kt & 3) == 2 ? L.z : L.w;
+      const uint32_t wh = (kt & 3) == 0 ? H.x : (kt & 3) == 1 ? H.y : (kt & 3) == 2 ? H.z : H.w;
+      uint32_t a[4];
+      e4m3x4_to_f16x2x2(wl, a[0], a[2]);
+      e4m3x4_to_f16x2x2(wh, a[1], a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        MmaOp<MmaT>::run((kt & 1) ? acc2[nt] : sacc[nt], a, qf[kt][nt][0], qf[kt][nt][1]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] += acc2[nt][e];
+  }
+  template <int NT>
+  __device__ static void pv(float (&o)[D / 16][NT][4], const uint8_t* sv, int mt,
+                            const uint32_t (&pb)[NT][2], int lane) {
+    const int c4 = lane & 3, r4 = lane >> 2;
+    const int t0 = mt * 16 + 2 * c4;  // token rows t0, t0+1, t0+8, t0+9
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int col = 32 * p + 4 * r4;
+      const uint32_t w0 = lds<uint32_t>(sv, t0, col), w1 = lds<uint32_t>(sv, t0 + 1, col);
+      const uint32_t w2 = lds<uint32_t>(sv, t0 + 8, col), w3 = lds<uint32_t>(sv, t0 + 9, col);
+      // bytes b of a word: (m-tile 2p, row r4), (2p, r4+8), (2p+1, r4), (2p+1, r4+8)
+      const uint32_t e01 = __byte_perm(w0, w1, 0x5140), o01 = __byte_perm(w0, w1, 0x7362);
+      const uint32_t e89 = __byte_perm(w2, w3, 0x5140), o89 = __byte_perm(w2, w3, 0x7362);
+      uint32_t ae[4], ao[4];
+      e4m3x4_to_f16x2x2(e01, ae[0], ae[1]);
+      e4m3x4_to_f16x2x2(e89, ae[2], ae[3]);
+      e4m3x4_to_f16x2x2(o01, ao[0], ao[1]);
+      e4m3x4_to_f16x2x2(o89, ao[2], ao[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        MmaOp<MmaT>::run(o[2 * p][nt], ae, pb[nt][0], pb[nt][1]);
+        MmaOp<MmaT>::run(o[2 * p + 1][nt], ao, pb[nt][0], pb[nt][1]);
+      }
+    }
+  }
+  __device__ static int out_d(int dt, int e, int r4) {
+    return 32 * (dt >> 1) + 4 * r4 + 2 * (dt & 1) + (e >> 1);
+  }
+};
+
+template <typename T, int BS>
+template <typename V>
+__device__ V E4m3Tiles<T, BS>::lds(const uint8_t* tile, int row, int col) {
+  const uint32_t a = sw128(smem_u32(tile), row, col);
+  if constexpr (sizeof(V) == 16) {
+    V v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+  } else {
+    V v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+  }
+}
+
+// --------------------------------------------------------------- kernel
+template <class Tiles, int BS, int NT>
 struct DecodeShape {
+  static constexpr int D = Tiles::D;
   static constexpr int NW = 4;                      // consumer warps
   static constexpr int THREADS = (NW + 1) * 32;     // + producer warp
-  static constexpr int HALVES = D / 64;             // 128-byte column groups
-  static constexpr int HALF_BYTES = BS * 128;       // one column group of a tile
-  static constexpr int TILE_BYTES = BS * D * 2;     // K or V tile of one (block, kv head)
+  static constexpr int TILE_BYTES = Tiles::TILE_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NS = (BS == 16) ? 8 : 4;     // ring depth
+  static constexpr int NS = Tiles::NS;              // ring depth
   static constexpr int RING_BYTES = NS * STAGE_BYTES;
   static constexpr int MERGE_BYTES = NW * (NT * 8) * (D + 2) * 4;
   static constexpr int BODY_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
   static constexpr int SMEM_BYTES = 1024 + BODY_BYTES + 2 * NS * 8;
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
-  static_assert(NS % NW == 0 || NW % NS == 0, "ring depth vs consumer warps");
+  static_assert(NS % NW == 0, "ring depth vs consumer warps");
 };
 
-template <typename T, int D, int BS, int NT>
-__global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
+template <class Tiles, int BS, int NT>
+__global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
-  using Shape = DecodeShape<T, D, BS, NT>;
-  constexpr int NW = Shape::NW, NS = Shape::NS, HALVES = Shape::HALVES;
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  using MmaT = typename Tiles::MmaT;
+  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS;
   constexpr int GP = NT * 8;  // padded heads per CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -134,13 +405,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
           if (i >= NS && alive) alive = mbar_wait(&empty_bar[st], ((i / NS) - 1) & 1);
           mbar_arrive_expect_tx(&full_bar[st], Shape::STAGE_BYTES);
           uint8_t* sk = smem + st * Shape::STAGE_BYTES;
-          uint8_t* sv = sk + Shape::TILE_BYTES;
-          const int row = (ph * p.num_kv_heads + kvh) * BS;
-#pragma unroll
-          for (int h = 0; h < HALVES; ++h) {
-            tma_load_2d(sk + h * Shape::HALF_BYTES, &tm_k, h * 64, row, &full_bar[st], policy);
-            tma_load_2d(sv + h * Shape::HALF_BYTES, &tm_v, h * 64, row, &full_bar[st], policy);
-          }
+          Tiles::issue(sk, sk + Shape::TILE_BYTES, &tm_k, &tm_v,
+                       (ph * p.num_kv_heads + kvh) * BS, &full_bar[st], policy);
         }
       }
     }
@@ -150,27 +416,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
   // -------------------------------------------------------------- consumers
   const int G = p.group;
   const int c4 = lane & 3, r4 = lane >> 2;
-  // Q^T as the B operand (k = head dim, n = query head of the group).
-  uint32_t qf[D / 16][NT][2];
-  {
-    const T* qbase = reinterpret_cast<const T*>(p.query) +
-                     ((size_t)s * p.num_q_heads + (size_t)kvh * G) * D;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int g = nt * 8 + r4;
-#pragma unroll
-      for (int kt = 0; kt < D / 16; ++kt) {
-        uint32_t b0 = 0, b1 = 0;
-        if (g < G) {
-          const uint32_t* row = reinterpret_cast<const uint32_t*>(qbase + (size_t)g * D);
-          b0 = __ldg(row + (kt * 16 + 2 * c4) / 2);
-          b1 = __ldg(row + (kt * 16 + 2 * c4 + 8) / 2);
-        }
-        qf[kt][nt][0] = b0;
-        qf[kt][nt][1] = b1;
-      }
-    }
-  }
+  uint32_t qf[D / 16][NT][2];  // Q^T as the B operand
+  Tiles::template load_q<NT>(
+      qf, reinterpret_cast<const T*>(p.query) + ((size_t)s * p.num_q_heads + (size_t)kvh * G) * D,
+      G, lane);
 
   float m_run[NT][2], l_run[NT][2];
   float o[D / 16][NT][4];
@@ -184,25 +433,22 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
       for (int e = 0; e < 4; ++e) o[dt][nt][e] = 0.f;
   }
 
-  const uint32_t smem_base = smem_u32(smem);
   bool alive = true;
   for (int i = warp; i < nblk; i += NW) {
     const int st = i % NS;
     if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1);
-    const uint32_t sk = smem_base + st * Shape::STAGE_BYTES;
-    const uint32_t sv = sk + Shape::TILE_BYTES;
+    const uint8_t* sk = smem + st * Shape::STAGE_BYTES;
+    const uint8_t* sv = sk + Shape::TILE_BYTES;
     const int tok_blk = (blk0 + i) * BS;  // logical position of the block's first slot
     const int valid = min(BS, L - tok_blk);
     if (valid < BS) {
       // Slots past the sequence end may hold anything (NaN included); zero
       // their V rows so that 0-weight x garbage cannot poison the PV product.
       uint8_t* v_gen = smem + st * Shape::STAGE_BYTES + Shape::TILE_BYTES;
-      for (int idx = lane; idx < (BS - valid) * HALVES * 8; idx += 32) {
-        const int r = valid + idx / (HALVES * 8), rem = idx % (HALVES * 8);
-        const int h = rem / 8, ch = rem % 8;
-        *reinterpret_cast<uint4*>(v_gen + h * Shape::HALF_BYTES + r * 128 + ch * 16) =
+      constexpr int CPR = Tiles::ZERO_CHUNKS_PER_ROW;
+      for (int idx = lane; idx < (BS - valid) * CPR; idx += 32)
+        *reinterpret_cast<uint4*>(Tiles::zero_chunk(v_gen, valid + idx / CPR, idx % CPR)) =
             make_uint4(0, 0, 0, 0);
-      }
       __syncwarp();
     }
 #pragma unroll
@@ -212,64 +458,61 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-      // S^T = K Q^T
-#pragma unroll
-      for (int kt = 0; kt < D / 16; ++kt) {
-        const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int chunk = (kt & 3) * 2 + (lane >> 4);
-        const uint32_t addr = sk + (kt >> 2) * Shape::HALF_BYTES + row * 128 +
-                              ((chunk ^ (row & 7)) << 4);
-        uint32_t a[4];
-        ldmatrix_x4(a, addr);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) MmaOp<T>::run(sacc[nt], a, qf[kt][nt][0], qf[kt][nt][1]);
-      }
+      Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
       // online softmax over this sub-tile's 16 tokens
       const int t_lo = tok_blk + mt * 16 + r4;
       const bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+      // The running max m_run is raised only when a sub-tile's max exceeds
+      // it by more than 8 (log2 units), so P <= 2^8 stays in 16-bit range and
+      // O is rescaled rarely; the stale max cancels in O / l.
       uint32_t pb[NT][2];
+      float sl[NT][2], sh[NT][2], alpha[NT][2];
+      bool raise = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          sl[nt][j] = ok_lo ? sacc[nt][j] * p.scale_log2 : -INFINITY;
+          sh[nt][j] = ok_hi ? sacc[nt][j + 2] * p.scale_log2 : -INFINITY;
+          float mx = fmaxf(sl[nt][j], sh[nt][j]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          alpha[nt][j] = 1.f;
+          if (mx > m_run[nt][j] + 8.f) {
+            alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);  // 0 when m_run is -inf
+            m_run[nt][j] = mx;
+            raise = true;
+          }
+        }
+      if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            l_run[nt][j] *= alpha[nt][j];
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+              o[dt][nt][j] *= alpha[nt][j];
+              o[dt][nt][j + 2] *= alpha[nt][j];
+            }
+          }
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float pv[4];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const float s_lo = ok_lo ? sacc[nt][j] * p.scale_log2 : -INFINITY;
-          const float s_hi = ok_hi ? sacc[nt][j + 2] * p.scale_log2 : -INFINITY;
-          float mx = fmaxf(s_lo, s_hi);
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float m_new = fmaxf(m_run[nt][j], mx);
-          const float m_use = m_new == -INFINITY ? 0.f : m_new;
-          const float alpha = exp2f(m_run[nt][j] - m_use);
-          pv[j] = exp2f(s_lo - m_use);
-          pv[j + 2] = exp2f(s_hi - m_use);
-          l_run[nt][j] = l_run[nt][j] * alpha + pv[j] + pv[j + 2];
-          m_run[nt][j] = m_new;
-#pragma unroll
-          for (int dt = 0; dt < D / 16; ++dt) {
-            o[dt][nt][j] *= alpha;
-            o[dt][nt][j + 2] *= alpha;
-          }
+          const float m_use = m_run[nt][j] == -INFINITY ? 0.f : m_run[nt][j];
+          pv[j] = ex2_approx(sl[nt][j] - m_use);
+          pv[j + 2] = ex2_approx(sh[nt][j] - m_use);
+          l_run[nt][j] += pv[j] + pv[j + 2];
         }
         // accumulator rows t / t+8, cols (g, g+1) -> B-operand layout of P^T
-        pb[nt][0] = movmatrix_trans(MmaOp<T>::pack(pv[0], pv[1]));
-        pb[nt][1] = movmatrix_trans(MmaOp<T>::pack(pv[2], pv[3]));
+        pb[nt][0] = movmatrix_trans(MmaOp<MmaT>::pack(pv[0], pv[1]));
+        pb[nt][1] = movmatrix_trans(MmaOp<MmaT>::pack(pv[2], pv[3]));
       }
-      // O^T += V^T P^T
-#pragma unroll
-      for (int dt = 0; dt < D / 16; ++dt) {
-        const int j = lane >> 3;
-        const int trow = mt * 16 + (lane & 7) + (j >> 1) * 8;
-        const int dcol = dt * 16 + (j & 1) * 8;
-        const int chunk = (dcol & 63) >> 3;
-        const uint32_t addr = sv + (dcol >> 6) * Shape::HALF_BYTES + trow * 128 +
-                              ((chunk ^ (trow & 7)) << 4);
-        uint32_t a[4];
-        ldmatrix_x4_trans(a, addr);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) MmaOp<T>::run(o[dt][nt], a, pb[nt][0], pb[nt][1]);
-      }
+      Tiles::template pv<NT>(o, sv, mt, pb, lane);
     }
     if (valid < BS) fence_proxy_async_smem();  // our zero stores precede the next TMA write
     __syncwarp();
@@ -296,9 +539,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
     for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int d = dt * 16 + r4 + (e >> 1) * 8;
         const int g = nt * 8 + 2 * c4 + (e & 1);
-        mg[(warp * GP + g) * RS + d] = o[dt][nt][e];
+        mg[(warp * GP + g) * RS + Tiles::out_d(dt, e, r4)] = o[dt][nt][e];
       }
   if (r4 == 0) {
 #pragma unroll
@@ -325,6 +567,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, NT>::THREADS, 2)
       num += sc * mg[(w * GP + g) * RS + d];
       den += sc * mg[(w * GP + g) * RS + D + 1];
     }
+    num *= p.v_scale;
     const int h = kvh * G + g;
     if (single) {
       const float v = den > 0.f ? num / den : 0.f;

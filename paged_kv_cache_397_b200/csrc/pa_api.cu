@@ -41,25 +41,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D row-major [rows][cols] 16-bit tensor with a row pitch of `pitch_elems`,
-// boxes of {64 columns, box_rows rows}, 128-byte swizzle.
+// 2-D row-major [rows][cols] tensor with a row pitch of `pitch_elems`, boxes of
+// {128 bytes of columns, box_rows rows}, 128-byte swizzle.
 bool make_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                  uint64_t pitch_elems, uint32_t box_rows, pa_dtype dt) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
+  const uint32_t esize = dt == PA_FP8_E4M3 ? 1 : 2;
+  const CUtensorMapDataType type = dt == PA_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {pitch_elems * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {pitch_elems * esize};
+  cuuint32_t box[2] = {128 / esize, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                  2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 bool valid_dtype(pa_dtype d) { return d == PA_F16 || d == PA_BF16; }
+bool valid_cache_dtype(pa_dtype d) { return valid_dtype(d) || d == PA_FP8_E4M3; }
 
 // Split-KV scratch for pa_decode_static_workspace, for callers that cannot
 // allocate: one array per device, part of the module's own device memory.
@@ -105,11 +108,12 @@ int partition_tokens_for(int requested, int num_seqs, int num_kv_heads, int bloc
   return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len);
 }
 
-template <typename T, int D, int BS, int NT>
+template <class Tiles, int BS, int NT>
 pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
                      int num_parts, cudaStream_t stream) {
-  using Shape = pa::DecodeShape<T, D, BS, NT>;
-  auto kern = pa::decode_kernel<T, D, BS, NT>;
+  using Shape = pa::DecodeShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  auto kern = pa::decode_kernel<Tiles, BS, NT>;
   static bool configured = false;  // per instantiation; attribute is per device-function
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -121,26 +125,37 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
   kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (num_parts > 1) {
-    pa::decode_reduce_kernel<T, D><<<p.num_seqs * p.num_q_heads, D, 0, stream>>>(p, BS);
+    pa::decode_reduce_kernel<T, Shape::D><<<p.num_seqs * p.num_q_heads, Shape::D, 0, stream>>>(
+        p, BS);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
 }
 
-template <typename T, int D, int BS>
+template <class Tiles, int BS>
 pa_status dispatch_group(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
                          int num_parts, cudaStream_t stream) {
-  if (p.group <= 8) return run_decode<T, D, BS, 1>(mk, mv, p, num_parts, stream);
-  return run_decode<T, D, BS, 2>(mk, mv, p, num_parts, stream);
+  if (p.group <= 8) return run_decode<Tiles, BS, 1>(mk, mv, p, num_parts, stream);
+  return run_decode<Tiles, BS, 2>(mk, mv, p, num_parts, stream);
 }
 
 template <typename T>
 pa_status dispatch_decode(int D, int BS, const CUtensorMap& mk, const CUtensorMap& mv,
                           pa::DecodeParams p, int num_parts, cudaStream_t stream) {
-  if (D == 128 && BS == 16) return dispatch_group<T, 128, 16>(mk, mv, p, num_parts, stream);
-  if (D == 128 && BS == 32) return dispatch_group<T, 128, 32>(mk, mv, p, num_parts, stream);
-  if (D == 64 && BS == 16) return dispatch_group<T, 64, 16>(mk, mv, p, num_parts, stream);
-  if (D == 64 && BS == 32) return dispatch_group<T, 64, 32>(mk, mv, p, num_parts, stream);
+  using namespace pa;
+  if (D == 128 && BS == 16) return dispatch_group<HalfTiles<T, 128, 16>, 16>(mk, mv, p, num_parts, stream);
+  if (D == 128 && BS == 32) return dispatch_group<HalfTiles<T, 128, 32>, 32>(mk, mv, p, num_parts, stream);
+  if (D == 64 && BS == 16) return dispatch_group<HalfTiles<T, 64, 16>, 16>(mk, mv, p, num_parts, stream);
+  if (D == 64 && BS == 32) return dispatch_group<HalfTiles<T, 64, 32>, 32>(mk, mv, p, num_parts, stream);
+  return PA_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+pa_status dispatch_decode_fp8(int BS, const CUtensorMap& mk, const CUtensorMap& mv,
+                              pa::DecodeParams p, int num_parts, cudaStream_t stream) {
+  using namespace pa;
+  if (BS == 16) return dispatch_group<E4m3Tiles<T, 16>, 16>(mk, mv, p, num_parts, stream);
+  if (BS == 32) return dispatch_group<E4m3Tiles<T, 32>, 32>(mk, mv, p, num_parts, stream);
   return PA_ERR_UNSUPPORTED;
 }
 
@@ -240,13 +255,15 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
                          int num_pairs, int num_kv_heads, int head_dim, int block_size,
                          int num_blocks, pa_dtype dtype, pa_stream_t stream) {
   if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-      num_blocks <= 0 || !valid_dtype(dtype))
+      num_blocks <= 0 || !valid_cache_dtype(dtype))
     return PA_ERR_INVALID_ARG;
   if (num_pairs == 0) return PA_OK;
   if (!key_cache || !value_cache || !block_pairs) return PA_ERR_INVALID_ARG;
   if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_INVALID_ARG;
-  if ((head_dim * 2) % 16 != 0) return PA_ERR_UNSUPPORTED;
-  const int64_t chunks = (int64_t)num_kv_heads * block_size * head_dim * 2 / 16;
+  const int64_t block_bytes =
+      (int64_t)num_kv_heads * block_size * head_dim * (dtype == PA_FP8_E4M3 ? 1 : 2);
+  if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+  const int64_t chunks = block_bytes / 16;
   pa::copy_blocks_kernel<8><<<dim3(num_pairs, 2), 256, 0, (cudaStream_t)stream>>>(
       reinterpret_cast<uint4*>(key_cache), reinterpret_cast<uint4*>(value_cache), block_pairs,
       chunks, num_blocks);
@@ -275,15 +292,25 @@ pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_hea
   return PA_OK;
 }
 
-pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
-                    const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int num_blocks, int max_blocks_per_seq, int max_seq_len,
-                    int partition_tokens, float scale, pa_dtype dtype, void* workspace,
-                    size_t workspace_bytes, pa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation, partition planning and launch shared by pa_decode (fp16 / bf16
+// caches) and pa_decode_fp8 (E4M3 caches, kv_fp8 = true).
+pa_status decode_impl(void* out, const void* query, const void* key_cache,
+                      const void* value_cache, const int32_t* block_tables,
+                      const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                      int max_seq_len, int partition_tokens, float scale, float k_scale,
+                      float v_scale, bool kv_fp8, pa_dtype dtype, void* workspace,
+                      size_t workspace_bytes, pa_stream_t stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
       max_blocks_per_seq <= 0 || max_seq_len < 0 || partition_tokens < 0 ||
       !valid_dtype(dtype) || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (kv_fp8 && !(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) &&
+                  v_scale > 0.f))
     return PA_ERR_INVALID_ARG;
   if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
@@ -296,6 +323,7 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
   if (num_seqs > 65535) return PA_ERR_INVALID_ARG;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (kv_fp8 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   const int group = num_q_heads / num_kv_heads;
   if (group > 16) return PA_ERR_UNSUPPORTED;
   if ((long long)num_blocks * num_kv_heads * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
@@ -311,8 +339,9 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
 
   CUtensorMap mk, mv;
   const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
-  if (!make_map_2d(&mk, key_cache, head_dim, rows, head_dim, block_size, dtype) ||
-      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, block_size, dtype))
+  const pa_dtype cache_dt = kv_fp8 ? PA_FP8_E4M3 : dtype;
+  if (!make_map_2d(&mk, key_cache, head_dim, rows, head_dim, block_size, cache_dt) ||
+      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, block_size, cache_dt))
     return PA_ERR_CUDA;
 
   pa::DecodeParams p;
@@ -333,11 +362,78 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.part_blocks = pt / block_size;
   p.max_parts = num_parts;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * (kv_fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+  p.v_scale = kv_fp8 ? v_scale : 1.f;
   auto st = (cudaStream_t)stream;
+  if (kv_fp8) {
+    if (dtype == PA_BF16) return dispatch_decode_fp8<__nv_bfloat16>(block_size, mk, mv, p, num_parts, st);
+    return dispatch_decode_fp8<__half>(block_size, mk, mv, p, num_parts, st);
+  }
   if (dtype == PA_BF16)
     return dispatch_decode<__nv_bfloat16>(head_dim, block_size, mk, mv, p, num_parts, st);
   return dispatch_decode<__half>(head_dim, block_size, mk, mv, p, num_parts, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, int max_seq_len,
+                    int partition_tokens, float scale, pa_dtype dtype, void* workspace,
+                    size_t workspace_bytes, pa_stream_t stream) {
+  return decode_impl(out, query, key_cache, value_cache, block_tables, seq_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                     max_blocks_per_seq, max_seq_len, partition_tokens, scale, 1.f, 1.f, false,
+                     dtype, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_fp8(void* out, const void* query, const uint8_t* key_cache,
+                        const uint8_t* value_cache, const int32_t* block_tables,
+                        const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                        int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                        int max_seq_len, int partition_tokens, float scale, float k_scale,
+                        float v_scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                        pa_stream_t stream) {
+  return decode_impl(out, query, key_cache, value_cache, block_tables, seq_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                     max_blocks_per_seq, max_seq_len, partition_tokens, scale, k_scale, v_scale,
+                     true, dtype, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, uint8_t* key_cache,
+                                   uint8_t* value_cache, const int64_t* slot_mapping,
+                                   int num_tokens, int num_kv_heads, int head_dim,
+                                   int block_size, int num_blocks, float k_scale, float v_scale,
+                                   pa_dtype dtype, pa_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || !valid_dtype(dtype) || !std::isfinite(k_scale) || k_scale <= 0.f ||
+      !std::isfinite(v_scale) || v_scale <= 0.f)
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if (head_dim % 16 != 0) return PA_ERR_UNSUPPORTED;
+  const long long total = (long long)num_tokens * num_kv_heads * (head_dim / 16);
+  const int threads = 256;
+  const long long grid = (total + threads - 1) / threads;
+  if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
+  const int64_t num_slots = (int64_t)num_blocks * block_size;
+  auto st = (cudaStream_t)stream;
+  if (dtype == PA_BF16)
+    pa::reshape_and_cache_fp8_kernel<__nv_bfloat16><<<(unsigned)grid, threads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(key), reinterpret_cast<const __nv_bfloat16*>(value),
+        key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+        num_slots, k_scale, v_scale);
+  else
+    pa::reshape_and_cache_fp8_kernel<__half><<<(unsigned)grid, threads, 0, st>>>(
+        reinterpret_cast<const __half*>(key), reinterpret_cast<const __half*>(value), key_cache,
+        value_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size, num_slots,
+        k_scale, v_scale);
+  return launch_status();
 }
 
 pa_status pa_decode_static_workspace(void* out, const void* query, const void* key_cache,

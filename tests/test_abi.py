@@ -22,7 +22,7 @@ def lib():
 def _declared():
     text = open(os.path.join(ROOT, "include", "pa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
@@ -35,7 +35,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", pa.lib_path], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (pa_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (pa_[a-z0-9_]+)\b", out))
     missing = [n for n in _declared() if n not in exported]
     assert not missing, f"declared but not exported: {missing}"
     assert sorted(pa.EXPORTED_SYMBOLS) == _declared()
