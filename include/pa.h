@@ -277,6 +277,69 @@ pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,
                            int max_blocks_per_seq, float scale, pa_dtype dtype,
                            pa_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Host block manager — the allocator that produces block tables, slot
+ * mappings and copy-on-write pairs for the kernels above.  Host memory only;
+ * no CUDA call.  "PagedAttention: KV cache as virtual memory", "Deep dive"
+ * (a block pool with an O(1) free queue in eviction order, per-block
+ * reference counts, a prefix cache keyed by the hash of a full block's tokens
+ * and its parent's key, allocate-on-append, free at count zero) and
+ * "PagedAttention: Why Static Batching Wastes Your KV Cache", "How does
+ * copy-on-write eliminate duplicate prompt KV cache?" (a sequence about to
+ * write into a shared block gets its own copy).  Not thread-safe: one
+ * manager per scheduler thread.  Sequence ids are caller-chosen int64.
+ * ------------------------------------------------------------------------ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* Pool of num_blocks blocks of block_size tokens; enable_prefix_caching != 0
+ * turns on full-block prefix sharing.  Blocks are handed out 0, 1, 2, ...
+ * while the pool is fresh. */
+pa_status pa_bm_create(int num_blocks, int block_size, int enable_prefix_caching,
+                       pa_block_manager **out);
+void pa_bm_destroy(pa_block_manager *bm);
+
+/* Admit a sequence with its prompt tokens: leading full blocks whose prefix
+ * key is cached are shared (reference count + 1, revived from the free queue
+ * if needed); the rest come from the front of the free queue.  Writes the
+ * number of prompt tokens whose K/V are already cached.  PA_ERR_OUT_OF_RANGE
+ * (state unchanged) when the pool cannot hold the prompt. */
+pa_status pa_bm_add_sequence(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens,
+                             int num_tokens, int *num_cached_tokens);
+
+/* Append generated tokens.  A new block is taken whenever the last one is
+ * full.  If the last block is partially filled and shared (count > 1), it is
+ * first replaced by a fresh block and the (src, dst) pair is queued for
+ * pa_bm_take_copies (copy-on-write).  PA_ERR_OUT_OF_RANGE (state unchanged)
+ * when the pool runs out. */
+pa_status pa_bm_append(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens,
+                       int num_tokens);
+
+/* The child shares every block of the parent (parallel sampling, beam search). */
+pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id);
+
+/* Finish a sequence: every block's count drops by one; blocks reaching zero
+ * go to the back of the free queue, last logical block first.  Cached full
+ * blocks keep their key until reused, so later prompts can still hit them. */
+pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id);
+
+/* The sequence's physical blocks in logical order into out[capacity] (the
+ * rest filled with -1); PA_ERR_WORKSPACE if capacity is too small. */
+pa_status pa_bm_block_table(const pa_block_manager *bm, int64_t seq_id, int32_t *out,
+                            int capacity, int *num_blocks);
+
+/* Slots of logical positions start .. start + count - 1 (physical * B + offset). */
+pa_status pa_bm_slots(const pa_block_manager *bm, int64_t seq_id, int start, int count,
+                      int64_t *out);
+
+/* Move the queued copy-on-write pairs into pairs[capacity][2] and return how
+ * many; returns minus the number pending (and takes none) if capacity is
+ * too small. */
+int pa_bm_take_copies(pa_block_manager *bm, int64_t *pairs, int capacity);
+
+int pa_bm_num_free_blocks(const pa_block_manager *bm);
+int pa_bm_ref_count(const pa_block_manager *bm, int block);
+int pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id); /* -1 if unknown */
+
 /*
  * pa_get_device_error — synchronise `stream`, then read and clear the device
  * error word of the current device (a bitwise OR of PA_DEVERR_* since the

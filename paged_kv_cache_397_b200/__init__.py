@@ -28,7 +28,7 @@ __all__ = [
     "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
-    "pa_reshape_and_cache_fp8", "pa_decode_fp8",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "BlockManager",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
 ]
@@ -61,6 +61,18 @@ _SIGS = {
     "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                               _i, _f, _i, _p]),
     "pa_get_device_error": (_i, [ctypes.POINTER(ctypes.c_uint), _p]),
+    "pa_bm_create": (_i, [_i, _i, _i, ctypes.POINTER(_p)]),
+    "pa_bm_destroy": (None, [_p]),
+    "pa_bm_add_sequence": (_i, [_p, ctypes.c_int64, _p, _i, ctypes.POINTER(_i)]),
+    "pa_bm_append": (_i, [_p, ctypes.c_int64, _p, _i]),
+    "pa_bm_fork": (_i, [_p, ctypes.c_int64, ctypes.c_int64]),
+    "pa_bm_free": (_i, [_p, ctypes.c_int64]),
+    "pa_bm_block_table": (_i, [_p, ctypes.c_int64, _p, _i, ctypes.POINTER(_i)]),
+    "pa_bm_slots": (_i, [_p, ctypes.c_int64, _i, _i, _p]),
+    "pa_bm_take_copies": (_i, [_p, _p, _i]),
+    "pa_bm_num_free_blocks": (_i, [_p]),
+    "pa_bm_ref_count": (_i, [_p, _i]),
+    "pa_bm_num_tokens": (_i, [_p, ctypes.c_int64]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGS)
 
@@ -332,3 +344,88 @@ def pa_get_device_error(stream=None) -> int:
     if st not in (PA_OK, PA_ERR_OUT_OF_RANGE):
         raise PAError("pa_get_device_error", st)
     return int(w.value)
+
+
+class BlockManager:
+    """Handle on the library's host block manager (include/pa.h, pa_bm_*).
+
+    Marshalling only: token ids in, block tables / slots / copy pairs out as
+    numpy arrays.  ``add_sequence`` / ``append`` raise PAError with
+    PA_ERR_OUT_OF_RANGE when the pool is exhausted (state unchanged).
+    """
+
+    def __init__(self, num_blocks: int, block_size: int, enable_prefix_caching: bool = True):
+        import numpy as np  # local: the rest of the binding needs only torch
+        self._np = np
+        h = ctypes.c_void_p()
+        _check("pa_bm_create", lib().pa_bm_create(int(num_blocks), int(block_size),
+                                                   int(bool(enable_prefix_caching)),
+                                                   ctypes.byref(h)))
+        self._h = h
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _tokens(self, tokens):
+        a = self._np.ascontiguousarray(tokens, dtype=self._np.int32)
+        return a, a.ctypes.data_as(ctypes.c_void_p)
+
+    def add_sequence(self, seq_id: int, tokens) -> int:
+        a, ptr = self._tokens(tokens)
+        cached = ctypes.c_int(0)
+        _check("pa_bm_add_sequence", lib().pa_bm_add_sequence(self._h, int(seq_id), ptr, a.size,
+                                                              ctypes.byref(cached)))
+        return int(cached.value)
+
+    def append(self, seq_id: int, tokens) -> None:
+        a, ptr = self._tokens(tokens)
+        _check("pa_bm_append", lib().pa_bm_append(self._h, int(seq_id), ptr, a.size))
+
+    def fork(self, parent_id: int, child_id: int) -> None:
+        _check("pa_bm_fork", lib().pa_bm_fork(self._h, int(parent_id), int(child_id)))
+
+    def free(self, seq_id: int) -> None:
+        _check("pa_bm_free", lib().pa_bm_free(self._h, int(seq_id)))
+
+    def block_table(self, seq_id: int, capacity: int = None):
+        n = ctypes.c_int(0)
+        lib().pa_bm_block_table(self._h, int(seq_id), None, 0, ctypes.byref(n))
+        cap = n.value if capacity is None else int(capacity)
+        out = self._np.empty(cap, dtype=self._np.int32)
+        _check("pa_bm_block_table", lib().pa_bm_block_table(
+            self._h, int(seq_id), out.ctypes.data_as(ctypes.c_void_p), cap, ctypes.byref(n)))
+        return out
+
+    def slots(self, seq_id: int, start: int, count: int):
+        out = self._np.empty(int(count), dtype=self._np.int64)
+        _check("pa_bm_slots", lib().pa_bm_slots(self._h, int(seq_id), int(start), int(count),
+                                                out.ctypes.data_as(ctypes.c_void_p)))
+        return out
+
+    def take_copies(self):
+        n = -lib().pa_bm_take_copies(self._h, None, 0)
+        n = max(n, 0)
+        out = self._np.empty((n, 2), dtype=self._np.int64)
+        got = lib().pa_bm_take_copies(self._h, out.ctypes.data_as(ctypes.c_void_p), n)
+        if got < 0:
+            raise RuntimeError("pa_bm_take_copies: capacity mismatch")
+        return out[:got]
+
+    @property
+    def num_free_blocks(self) -> int:
+        return int(lib().pa_bm_num_free_blocks(self._h))
+
+    def ref_count(self, block: int) -> int:
+        return int(lib().pa_bm_ref_count(self._h, int(block)))
+
+    def num_tokens(self, seq_id: int) -> int:
+        return int(lib().pa_bm_num_tokens(self._h, int(seq_id)))

@@ -1,7 +1,8 @@
 """Build step for libpa.so: one nvcc invocation for sm_100a, in-tree.
 
 ``python -m paged_kv_cache_397_b200._build`` (or ``__graft_entry__.build()``)
-compiles ``csrc/pa_api.cu`` (which includes every kernel) into
+compiles ``csrc/pa_api.cu`` (which includes every kernel) and the host block
+manager ``csrc/block_manager.cpp`` into
 ``paged_kv_cache_397_b200/libpa.so``.  The CUDA runtime is linked statically
 and the driver is reached through ``cudaGetDriverEntryPoint``, so the library
 loads (and its symbols can be listed) on a machine without a GPU.
@@ -15,7 +16,7 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "pa_api.cu")
+SRCS = [os.path.join(PKG, "csrc", "pa_api.cu"), os.path.join(PKG, "csrc", "block_manager.cpp")]
 LIB = os.path.join(PKG, "libpa.so")
 DEPS = [os.path.join(PKG, "csrc", f) for f in os.listdir(os.path.join(PKG, "csrc"))] + [
     os.path.join(ROOT, "include", "pa.h")]
@@ -47,7 +48,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-o", tmp, SRC]
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-o", tmp, *SRCS]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)

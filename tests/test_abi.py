@@ -39,6 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
     missing = [n for n in _declared() if n not in exported]
     assert not missing, f"declared but not exported: {missing}"
     assert sorted(pa.EXPORTED_SYMBOLS) == _declared()
+    assert "pa_bm_create" in _declared()
     for n in _declared():
         assert hasattr(lib, n)
 
