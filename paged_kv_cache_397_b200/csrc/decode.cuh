@@ -177,9 +177,9 @@ struct HalfTiles {
 // Q K^T contracts over the head dim in the permuted order d = 32c + 4kt + j
 // (c = lane % 4, kt = k-step, j = 0..3), so lane c reads bytes [32c, 32c+32)
 // of a K row with two 16-byte loads.  O^T keeps head-dim rows in the permuted
-// order d = 32p + 4r + b (p = m-tile pair, r = lane / 4, b = byte), so the
-// V^T fragments come from one 4-byte word per token row; byte_perm pairs two
-// token rows along the contraction (token) axis.
+// order d = 16r + 4p + b (r = lane / 4, p = m-tile pair, b = byte), so the
+// V^T fragments of a 16-token sub-tile come from one 16-byte load per token
+// row; byte_perm pairs two token rows along the contraction (token) axis.
 template <typename T, int BS>
 struct E4m3Tiles {
   using Elem = T;
@@ -278,12 +278,17 @@ struct E4m3Tiles {
                             const uint32_t (&pb)[NT][2], int lane) {
     const int c4 = lane & 3, r4 = lane >> 2;
     const int t0 = mt * 16 + 2 * c4;  // token rows t0, t0+1, t0+8, t0+9
+    // bytes [16 r, 16 r + 16) of each of the four rows: word p, byte b holds
+    // head dim 16 r + 4 p + b = (m-tile 2p, row r), (2p, r+8), (2p+1, r), (2p+1, r+8)
+    const uint4 v0 = lds<uint4>(sv, t0, 16 * r4), v1 = lds<uint4>(sv, t0 + 1, 16 * r4);
+    const uint4 v8 = lds<uint4>(sv, t0 + 8, 16 * r4), v9 = lds<uint4>(sv, t0 + 9, 16 * r4);
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const int col = 32 * p + 4 * r4;
-      const uint32_t w0 = lds<uint32_t>(sv, t0, col), w1 = lds<uint32_t>(sv, t0 + 1, col);
-      const uint32_t w2 = lds<uint32_t>(sv, t0 + 8, col), w3 = lds<uint32_t>(sv, t0 + 9, col);
-      // bytes b of a word: (m-tile 2p, row r4), (2p, r4+8), (2p+1, r4), (2p+1, r4+8)
+      const uint32_t w0 = p == 0 ? v0.x : p == 1 ? v0.y : p == 2 ? v0.z : v0.w;
+      const uint32_t w1 = p == 0 ? v1.x : p == 1 ? v1.y : p == 2 ? v1.z : v1.w;
+      const uint32_t w2 = p == 0 ? v8.x : p == 1 ? v8.y : p == 2 ? v8.z : v8.w;
+      const uint32_t w3 = p == 0 ? v9.x : p == 1 ? v9.y : p == 2 ? v9.z : v9.w;
+      // pair the two token rows byte by byte (contraction runs along tokens)
       const uint32_t e01 = __byte_perm(w0, w1, 0x5140), o01 = __byte_perm(w0, w1, 0x7362);
       const uint32_t e89 = __byte_perm(w2, w3, 0x5140), o89 = __byte_perm(w2, w3, 0x7362);
       uint32_t ae[4], ao[4];
@@ -299,7 +304,7 @@ struct E4m3Tiles {
     }
   }
   __device__ static int out_d(int dt, int e, int r4) {
-    return 32 * (dt >> 1) + 4 * r4 + 2 * (dt & 1) + (e >> 1);
+    return 16 * r4 + 4 * (dt >> 1) + 2 * (dt & 1) + (e >> 1);
   }
 };
 
