@@ -10,7 +10,9 @@ Printed (rank 0, one JSON line): the decode KV bandwidth over the whole step
 (GB/s of algorithmic K/V bytes), decode tokens/s, the roofline of pa_decode,
 the prefill-chunk TFLOP/s of the 8 x 512-token chunk workload, an end-to-end
 figure through the C ABI with host buffers, clocks seen during the timed
-region, and the CPU oracle as a baseline.
+region, the CPU oracle as a baseline, and (single GPU) secondary figures: the
+same decode step over an FP8 pool, copy-on-write block copies and swap
+bandwidth to / from pinned host memory.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 For N > 1 launch with torch.distributed.run; every rank decodes its own batch
@@ -253,6 +255,72 @@ def prefill_measure(dev, steps, warmup, block_size):
             "tflops": flops / ms / 1e9, "causal_flop": flops}
 
 
+def fp8_decode_measure(dev, steps, warmup, hbm_peak):
+    """The same GQA decode step over an FP8 (E4M3) pool: slot mapping, FP8
+    append, FP8 decode.  GB/s of FP8 K/V bytes read."""
+    import paged_kv_cache_397_b200 as pa
+    w = synth.llama3_8b_gqa_decode_fp8()
+    kc, vc, bt = w.key_cache.to(dev), w.value_cache.to(dev), w.block_tables.to(dev)
+    ctx = w.context_lens.to(dev)
+    lens = (w.context_lens + 1).to(dev)
+    q, nk, nv = w.query.to(dev), w.new_key.to(dev), w.new_value.to(dev)
+    slots = torch.empty(w.num_seqs, dtype=torch.int64, device=dev)
+    out = torch.empty_like(q)
+    max_len = int(lens.max())
+    need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                       w.block_size, max_len)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        pa.pa_slot_mapping(slots, bt, ctx, w.block_size)
+        pa.pa_reshape_and_cache_fp8(nk, nv, kc, vc, slots, w.kv_scale, w.kv_scale)
+        pa.pa_decode_fp8(out, q, kc, vc, bt, lens, max_len, w.scale, w.kv_scale, w.kv_scale,
+                         workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ms = time_steps(step, steps, torch.cuda.current_stream()) / steps
+    kv = 2 * w.num_kv_heads * w.head_dim * int(lens.sum())
+    return {"workload": w.name, "ms_per_step": ms, "value": kv / ms / 1e6, "unit": "GB/s",
+            "hbm_frac": kv / ms / 1e6 / hbm_peak, "decode_tokens_per_s": w.num_seqs / ms * 1e3,
+            "kv_bytes_per_step": kv}
+
+
+def copy_and_swap_measure(dev, steps):
+    """Copy-on-write of the shared-prefix workload (128 block pairs) and swap
+    of 256 blocks of the GQA decode shape out to pinned host memory and back."""
+    import paged_kv_cache_397_b200 as pa
+    res = {}
+    w = synth.shared_prefix_cow()
+    kc, vc = w.key_cache.to(dev), w.value_cache.to(dev)
+    src = w.shared_blocks[w.cow_logical_block].repeat(w.num_seqs)
+    pairs = torch.stack([src, w.cow_dst_blocks], 1).to(torch.int64).to(dev)
+    fn = lambda: pa.pa_copy_blocks(kc, vc, pairs)
+    for _ in range(3):
+        fn()
+    ms = time_steps(fn, steps, torch.cuda.current_stream()) / steps
+    moved = 2 * 2 * pairs.shape[0] * kc[0].numel() * kc.element_size()  # K+V, read+write
+    res["copy_blocks"] = {"workload": w.name, "pairs": int(pairs.shape[0]), "us": ms * 1e3,
+                          "GBps_read_plus_write": moved / ms / 1e6}
+    del kc, vc
+    shape = (256, 8, 16, 128)
+    dk = torch.randn(shape, dtype=torch.float32, device=dev).to(torch.bfloat16)
+    dv = torch.randn(shape, dtype=torch.float32, device=dev).to(torch.bfloat16)
+    hk = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    ident = torch.stack([torch.arange(256), torch.arange(256)], 1).to(torch.int64).to(dev)
+    block_bytes = 2 * dk[0].numel() * dk.element_size()  # K + V
+    for name, f in (("swap_out_d2h", lambda: pa.pa_swap_blocks(hk, hv, dk, dv, ident)),
+                    ("swap_in_h2d", lambda: pa.pa_swap_blocks(dk, dv, hk, hv, ident))):
+        for _ in range(3):
+            f()
+        ms = time_steps(f, max(3, steps // 4), torch.cuda.current_stream()) / max(3, steps // 4)
+        res[name] = {"blocks": 256, "bytes": 256 * block_bytes, "us": ms * 1e3,
+                     "GBps": 256 * block_bytes / ms / 1e6}
+    return res
+
+
 def cpu_baseline(w, budget_s=10.0):
     """The oracle, as it stands, on a seeded sample of the batch's sequences."""
     import threadpoolctl
@@ -364,6 +432,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the FP8 decode, copy-on-write and swap measurements")
     ap.add_argument("--min-warmup-s", type=float, default=1.0,
                     help="keep warming up for at least this long so clocks settle")
     args = ap.parse_args()
@@ -443,6 +513,14 @@ def main():
             r["peak_kind"] = f"bf16 dense, {peak_kind} (burst)"
             prefill.append(r)
 
+    secondary = None
+    if world == 1 and not args.no_secondary:
+        torch.cuda.empty_cache()
+        secondary = {"fp8_decode": fp8_decode_measure(dev, steps=50, warmup=5,
+                                                      hbm_peak=hbm_peak)}
+        torch.cuda.empty_cache()
+        secondary.update(copy_and_swap_measure(dev, steps=50))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -463,6 +541,7 @@ def main():
                          "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
                          "peak_kind": f"hbm copy, {peak_kind}"},
             "prefill_chunk": prefill,
+            "secondary": secondary,
             "e2e": {"value": e2e_value, "unit": "GB/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,

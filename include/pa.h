@@ -130,6 +130,26 @@ pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int64_t *bloc
                          int num_blocks, pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_swap_blocks — copy whole blocks between two pools, e.g. out to a pool in
+ * host memory and back.  "PagedAttention: Why Static Batching Wastes Your KV
+ * Cache", "What happens when the GPU runs out of KV blocks?" (swapping:
+ * evicted blocks go to CPU RAM over PCIe and come back when the sequence is
+ * rescheduled).  For each pair (src, dst): dst pool block dst = src pool
+ * block src, for K and V (bit copy), all pairs in one kernel launch.
+ *   dst_key_cache, dst_value_cache  out  T[dst_num_blocks][num_kv_heads][block_size][head_dim]
+ *   src_key_cache, src_value_cache  in   T[src_num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_pairs                     in   int64[num_pairs][2] = {src, dst}, device memory
+ * Either pool may be pinned host memory (cudaHostAlloc / page-locked memory,
+ * which the GPU addresses through unified virtual addressing); the other is
+ * device memory.  dst ids must be distinct.  A pair with an id outside its
+ * pool is skipped and sets PA_DEVERR_BLOCK_RANGE.
+ */
+pa_status pa_swap_blocks(void *dst_key_cache, void *dst_value_cache, const void *src_key_cache,
+                         const void *src_value_cache, const int64_t *block_pairs, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int src_num_blocks,
+                         int dst_num_blocks, pa_dtype dtype, pa_stream_t stream);
+
+/*
  * pa_reshape_and_cache_fp8 — pa_reshape_and_cache into FP8 (E4M3) caches.
  *   "PagedAttention: KV cache as virtual memory", "Deep dive" and
  *   "Interviewer follow-ups" (an FP8 KV cache halves the bytes per block and

@@ -41,7 +41,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "logical_positions_to_slots", "reshape_and_cache", "copy_blocks",
+    "logical_positions_to_slots", "reshape_and_cache", "copy_blocks", "swap_blocks",
     "gather_logical", "attention", "paged_decode", "paged_prefill_chunk",
     "partial_attention", "combine_partials",
 ]
@@ -101,6 +101,18 @@ def copy_blocks(key_cache, value_cache, block_pairs):
     for src, dst in np.asarray(block_pairs, dtype=np.int64).reshape(-1, 2):
         key_cache[dst] = key_cache[src]
         value_cache[dst] = value_cache[src]
+
+
+def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, block_pairs):
+    """Swap: ``dst_pool[dst] = src_pool[src]`` for K and V, a bit copy between
+    two pools (device and host).
+
+    [Static] "What happens when the GPU runs out of KV blocks?": swapped-out
+    blocks are copied to CPU memory and copied back when the sequence resumes.
+    """
+    for src, dst in np.asarray(block_pairs, dtype=np.int64).reshape(-1, 2):
+        dst_key_cache[dst] = src_key_cache[src]
+        dst_value_cache[dst] = src_value_cache[src]
 
 
 # ---------------------------------------------------------------------------

@@ -28,7 +28,7 @@ __all__ = [
     "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
-    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "BlockManager",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "BlockManager",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
 ]
@@ -56,6 +56,7 @@ _SIGS = {
     "pa_decode_static_workspace": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                                         _i, _i, _f, _i, _p]),
     "pa_reshape_and_cache_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _i, _p]),
+    "pa_swap_blocks": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
     "pa_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _f,
                            _f, _i, _p, _sz, _p]),
     "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
@@ -243,6 +244,32 @@ def pa_decode_fp8(out, query, key_cache, value_cache, block_tables, seq_lens, ma
         int(block_tables.shape[1]), int(max_seq_len), int(partition_tokens), float(scale),
         float(k_scale), float(v_scale), _dtype_code(query), ws_ptr, ws_bytes, _stream(stream)))
     return out
+
+
+def _pool_ptr(t, name):
+    """A CUDA tensor, or a pinned CPU tensor (addressed by the GPU through UVA)."""
+    if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor")
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    return t.data_ptr()
+
+
+def pa_swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, block_pairs,
+                   stream=None):
+    """Copy blocks pairs[i][0] of the src pool to pairs[i][1] of the dst pool (K and V);
+    either pool may be pinned host memory (swap out / swap in)."""
+    snb, hkv, bs, d = _cache_dims(src_key_cache, src_value_cache)
+    dnb, hkv2, bs2, d2 = _cache_dims(dst_key_cache, dst_value_cache)
+    if (hkv, bs, d) != (hkv2, bs2, d2) or src_key_cache.dtype != dst_key_cache.dtype:
+        raise ValueError("source and destination pools differ in block shape or dtype")
+    if block_pairs.dim() != 2 or block_pairs.shape[1] != 2:
+        raise ValueError("block_pairs must be int64 [num_pairs][2]")
+    _check("pa_swap_blocks", lib().pa_swap_blocks(
+        _pool_ptr(dst_key_cache, "dst_key_cache"), _pool_ptr(dst_value_cache, "dst_value_cache"),
+        _pool_ptr(src_key_cache, "src_key_cache"), _pool_ptr(src_value_cache, "src_value_cache"),
+        _ptr(block_pairs, "block_pairs", torch.int64, 2), int(block_pairs.shape[0]), hkv, d, bs,
+        snb, dnb, _dtype_code(src_key_cache, allow_fp8=True), _stream(stream)))
 
 
 def pa_decode_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len) -> int:

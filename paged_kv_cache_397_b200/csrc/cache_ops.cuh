@@ -160,4 +160,35 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Block copies between two pools (swap out to / in from host memory).  One
+// CTA per (pair, K-or-V); either pool may be pinned host memory mapped into
+// the GPU's address space, so the loads or the stores cross PCIe / C2C; all
+// of a thread's loads are issued before its stores to keep many in flight.
+template <int kPerThread>
+__global__ void __launch_bounds__(256)
+    swap_blocks_kernel(uint4* dst_k, uint4* dst_v, const uint4* src_k, const uint4* src_v,
+                       const int64_t* __restrict__ pairs, int64_t chunks_per_block,
+                       int src_blocks, int dst_blocks) {
+  const int64_t src = pairs[2 * blockIdx.x], dst = pairs[2 * blockIdx.x + 1];
+  if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+    if (threadIdx.x == 0) record_error(PA_DEVERR_BLOCK_RANGE);
+    return;
+  }
+  const uint4* from = (blockIdx.y == 0 ? src_k : src_v) + src * chunks_per_block;
+  uint4* to = (blockIdx.y == 0 ? dst_k : dst_v) + dst * chunks_per_block;
+  for (int64_t base = 0; base < chunks_per_block; base += (int64_t)kPerThread * 256) {
+    uint4 r[kPerThread];
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int64_t i = base + (int64_t)k * 256 + threadIdx.x;
+      if (i < chunks_per_block) r[k] = from[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int64_t i = base + (int64_t)k * 256 + threadIdx.x;
+      if (i < chunks_per_block) to[i] = r[k];
+    }
+  }
+}
+
 }  // namespace pa

@@ -270,6 +270,29 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
   return launch_status();
 }
 
+pa_status pa_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_key_cache,
+                         const void* src_value_cache, const int64_t* block_pairs, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int src_num_blocks,
+                         int dst_num_blocks, pa_dtype dtype, pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      src_num_blocks <= 0 || dst_num_blocks <= 0 || !valid_cache_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || !block_pairs)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(dst_key_cache) || !aligned16(dst_value_cache) || !aligned16(src_key_cache) ||
+      !aligned16(src_value_cache))
+    return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes =
+      (int64_t)num_kv_heads * block_size * head_dim * (dtype == PA_FP8_E4M3 ? 1 : 2);
+  if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+  pa::swap_blocks_kernel<8><<<dim3(num_pairs, 2), 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<uint4*>(dst_key_cache), reinterpret_cast<uint4*>(dst_value_cache),
+      reinterpret_cast<const uint4*>(src_key_cache), reinterpret_cast<const uint4*>(src_value_cache),
+      block_pairs, block_bytes / 16, src_num_blocks, dst_num_blocks);
+  return launch_status();
+}
+
 int pa_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_seq_len) {
   if (num_seqs <= 0 || num_kv_heads <= 0 || block_size <= 0 || max_seq_len < 0) return 0;
   return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len);

@@ -98,3 +98,22 @@ def test_copy_blocks_bits():
     others = np.setdiff1d(np.arange(kc.shape[0]), dst)
     np.testing.assert_array_equal(kc[others], k0[others])
     np.testing.assert_array_equal(vc[others], v0[others])
+
+
+def test_swap_blocks_copies_between_pools_only_the_listed_blocks():
+    rng = np.random.default_rng(8)
+    dev_k = rng.integers(-5000, 5000, (10, 2, 16, 8)).astype(np.int16)
+    dev_v = rng.integers(-5000, 5000, (10, 2, 16, 8)).astype(np.int16)
+    host_k = np.zeros((4, 2, 16, 8), np.int16)
+    host_v = np.zeros((4, 2, 16, 8), np.int16)
+    pairs = np.array([[7, 0], [2, 3], [9, 1]])
+    oracle.swap_blocks(host_k, host_v, dev_k, dev_v, pairs)      # swap out
+    for s, d in pairs:
+        np.testing.assert_array_equal(host_k[d], dev_k[s])
+        np.testing.assert_array_equal(host_v[d], dev_v[s])
+    assert not host_k[2].any() and not host_v[2].any()
+    back_k, back_v = np.zeros_like(dev_k), np.zeros_like(dev_v)
+    oracle.swap_blocks(back_k, back_v, host_k, host_v, pairs[:, ::-1])  # swap back in
+    for s, _ in pairs:
+        np.testing.assert_array_equal(back_k[s], dev_k[s])
+        np.testing.assert_array_equal(back_v[s], dev_v[s])
