@@ -3,8 +3,9 @@
 One step = one decode iteration of the Llama-3-8B-shaped GQA batch (256
 sequences, 32 q / 8 kv heads, head_dim 128, bf16, 16-token blocks, lengths
 uniform in [128, 4096], shuffled physical blocks): slot mapping of the new
-token of every sequence, reshape_and_cache of its K/V, split-KV paged decode
-and the log-sum-exp reduce — all through libpa.so's C ABI.
+token of every sequence and the scatter of its K/V (one fused launch,
+pa_append), split-KV paged decode and the log-sum-exp reduce — all through
+libpa.so's C ABI.
 
 Printed (rank 0, one JSON line): the decode KV bandwidth over the whole step
 (GB/s of algorithmic K/V bytes), decode tokens/s, the roofline of pa_decode,
@@ -183,7 +184,7 @@ class DecodeStep:
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
         self.num_parts = math.ceil(self.max_len / pa.pa_decode_partition_tokens(
             w.num_seqs, w.num_kv_heads, w.block_size, self.max_len))
-        self.launches_per_step = 3 + (1 if self.num_parts > 1 else 0)
+        self.launches_per_step = 2 + (1 if self.num_parts > 1 else 0)
         total = int(self.lens.sum())
         self.kv_bytes = 2 * w.num_kv_heads * w.head_dim * 2 * total  # K and V, bf16
         # host-side copies for the end-to-end leg (pinned)
@@ -199,9 +200,8 @@ class DecodeStep:
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
 
     def append(self):
-        pa, w = self.pa, self.w
-        pa.pa_slot_mapping(self.slots, self.bt, self.ctx, w.block_size)
-        pa.pa_reshape_and_cache(self.nk, self.nv, self.kc, self.vc, self.slots)
+        # slot mapping + scatter of the new token, fused in one launch
+        self.pa.pa_append(self.nk, self.nv, self.kc, self.vc, self.bt, self.ctx)
 
     def decode(self):
         self.pa.pa_decode(self.out, self.q, self.kc, self.vc, self.bt, self.lens, self.max_len,

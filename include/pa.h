@@ -113,6 +113,21 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *key_cac
                                pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_append — pa_slot_mapping and pa_reshape_and_cache fused into one launch:
+ * each new token's slot is computed from block_tables / cu_q_lens / ctx_lens
+ * (same rule as pa_slot_mapping) and its K and V rows are written there (bit
+ * copy).  slot_mapping (int64[num_tokens]) receives the slots when non-NULL.
+ * Same layouts and argument meanings as the two calls it fuses; a position
+ * past the table sets PA_DEVERR_SEQ_RANGE and a table entry outside the pool
+ * PA_DEVERR_BLOCK_RANGE (the token is skipped, its slot reported as -1).
+ */
+pa_status pa_append(const void *key, const void *value, void *key_cache, void *value_cache,
+                    const int32_t *block_tables, const int32_t *cu_q_lens, const int32_t *ctx_lens,
+                    int64_t *slot_mapping, int num_seqs, int num_tokens, int max_blocks_per_seq,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                    pa_stream_t stream);
+
+/*
  * pa_copy_blocks — copy-on-write duplication of whole physical blocks.
  *   "PagedAttention: Why Static Batching Wastes Your KV Cache", "How does
  *   copy-on-write eliminate duplicate prompt KV cache?" (copy just that block

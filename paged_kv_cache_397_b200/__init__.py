@@ -28,7 +28,7 @@ __all__ = [
     "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
-    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "BlockManager",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_append", "BlockManager",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
 ]
@@ -48,6 +48,7 @@ _SIGS = {
     "pa_version": (_i, []),
     "pa_slot_mapping": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p]),
     "pa_reshape_and_cache": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]),
+    "pa_append": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]),
     "pa_copy_blocks": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p]),
     "pa_decode_partition_tokens": (_i, [_i, _i, _i, _i]),
     "pa_decode_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
@@ -187,6 +188,29 @@ def pa_reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, strea
         _ptr(key, "key"), _ptr(value, "value"), _ptr(key_cache, "key_cache"),
         _ptr(value_cache, "value_cache"), _ptr(slot_mapping, "slot_mapping", torch.int64, 1),
         int(key.shape[0]), hkv, d, bs, nb, _dtype_code(key_cache), _stream(stream)))
+
+
+def pa_append(key, value, key_cache, value_cache, block_tables, ctx_lens, cu_q_lens=None,
+              slot_mapping=None, stream=None):
+    """Slot mapping and K/V scatter of new tokens in one launch (include/pa.h)."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if key.shape != value.shape or key.dim() != 3 or tuple(key.shape[1:]) != (hkv, d):
+        raise ValueError("key/value must be [num_tokens][num_kv_heads][head_dim] like the cache")
+    if key.dtype != key_cache.dtype or value.dtype != key_cache.dtype:
+        raise ValueError("key/value dtype must match the cache")
+    S = int(ctx_lens.numel())
+    if block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("block_tables must be [num_seqs][max_blocks_per_seq]")
+    if cu_q_lens is not None and cu_q_lens.numel() != S + 1:
+        raise ValueError("cu_q_lens must have num_seqs + 1 entries")
+    if slot_mapping is not None and slot_mapping.numel() != key.shape[0]:
+        raise ValueError("slot_mapping needs one entry per token")
+    _check("pa_append", lib().pa_append(
+        _ptr(key, "key"), _ptr(value, "value"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(cu_q_lens, "cu_q_lens", torch.int32, 1), _ptr(ctx_lens, "ctx_lens", torch.int32, 1),
+        _ptr(slot_mapping, "slot_mapping", torch.int64, 1), S, int(key.shape[0]),
+        int(block_tables.shape[1]), hkv, d, bs, nb, _dtype_code(key_cache), _stream(stream)))
 
 
 def pa_copy_blocks(key_cache, value_cache, block_pairs, stream=None):

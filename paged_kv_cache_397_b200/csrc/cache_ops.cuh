@@ -44,6 +44,77 @@ __global__ void slot_mapping_kernel(int64_t* __restrict__ slots,
   slots[t] = (int64_t)phys * block_size + (pos % block_size);
 }
 
+// Slot of new token t: the slot-mapping rule above, shared by the fused
+// append kernel (one thread per 16-byte chunk recomputes it; the table and
+// lengths are tiny and cached).
+__device__ __forceinline__ int64_t new_token_slot(const int32_t* __restrict__ block_tables,
+                                                  const int32_t* __restrict__ cu,
+                                                  const int32_t* __restrict__ ctx_lens,
+                                                  int num_seqs, int t, int max_blocks_per_seq,
+                                                  int block_size) {
+  int s = t, off = 0;
+  if (cu != nullptr) {
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(cu + mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+    off = t - __ldg(cu + s);
+  }
+  const int pos = __ldg(ctx_lens + s) + off;
+  const int blk = pos / block_size;
+  if (pos < 0 || blk >= max_blocks_per_seq) return -2;  // past the table
+  return (int64_t)__ldg(block_tables + (size_t)s * max_blocks_per_seq + blk) * block_size +
+         (pos % block_size);
+}
+
+// Fused append (slot mapping + reshape_and_cache in one launch): one thread
+// per 16-byte chunk of one (token, kv head) row of K and of V; the first
+// chunk of each token also stores its slot when `slots_out` is given.
+template <int D>
+__global__ void append_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                              uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
+                              const int32_t* __restrict__ block_tables,
+                              const int32_t* __restrict__ cu, const int32_t* __restrict__ ctx_lens,
+                              int64_t* __restrict__ slots_out, int num_seqs, int num_tokens,
+                              int num_kv_heads, int max_blocks_per_seq, int block_size,
+                              int num_blocks) {
+  constexpr int CH = D * 2 / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)num_tokens * num_kv_heads * CH;
+  if (idx >= total) return;
+  const int c = (int)(idx % CH);
+  const int64_t th = idx / CH;
+  const int h = (int)(th % num_kv_heads);
+  const int t = (int)(th / num_kv_heads);
+  int64_t slot = new_token_slot(block_tables, cu, ctx_lens, num_seqs, t, max_blocks_per_seq,
+                                block_size);
+  const bool first = c == 0 && h == 0;
+  if (slot == -2) {
+    if (first) {
+      record_error(PA_DEVERR_SEQ_RANGE);
+      if (slots_out) slots_out[t] = -1;
+    }
+    return;
+  }
+  if (slot < 0 || slot >= (int64_t)num_blocks * block_size) {
+    if (first) {
+      record_error(PA_DEVERR_BLOCK_RANGE);
+      if (slots_out) slots_out[t] = -1;
+    }
+    return;
+  }
+  if (first && slots_out) slots_out[t] = slot;
+  const int64_t b = slot / block_size, off = slot % block_size;
+  const int64_t dst = ((b * num_kv_heads + h) * block_size + off) * CH + c;
+  const int64_t src = th * CH + c;
+  const uint4 kv = __ldg(key + src);
+  const uint4 vv = __ldg(value + src);
+  key_cache[dst] = kv;
+  value_cache[dst] = vv;
+}
+
 // One thread per 16-byte chunk of one (token, kv head) row of K and of V.
 template <int D>
 __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,

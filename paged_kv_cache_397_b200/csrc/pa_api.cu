@@ -251,6 +251,44 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* key_cac
   return launch_status();
 }
 
+pa_status pa_append(const void* key, const void* value, void* key_cache, void* value_cache,
+                    const int32_t* block_tables, const int32_t* cu_q_lens, const int32_t* ctx_lens,
+                    int64_t* slot_mapping, int num_seqs, int num_tokens, int max_blocks_per_seq,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                    pa_stream_t stream) {
+  if (num_tokens < 0 || num_seqs < 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 ||
+      head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (num_seqs == 0 || !key || !value || !key_cache || !value_cache || !block_tables ||
+      !ctx_lens)
+    return PA_ERR_INVALID_ARG;
+  if (cu_q_lens == nullptr && num_tokens != num_seqs) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  const long long total = (long long)num_tokens * num_kv_heads * (head_dim * 2 / 16);
+  const int threads = 256;
+  const long long grid = (total + threads - 1) / threads;
+  if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
+  auto st = (cudaStream_t)stream;
+  auto k = reinterpret_cast<const uint4*>(key);
+  auto v = reinterpret_cast<const uint4*>(value);
+  auto kc = reinterpret_cast<uint4*>(key_cache);
+  auto vc = reinterpret_cast<uint4*>(value_cache);
+  if (head_dim == 128)
+    pa::append_kernel<128><<<(unsigned)grid, threads, 0, st>>>(
+        k, v, kc, vc, block_tables, cu_q_lens, ctx_lens, slot_mapping, num_seqs, num_tokens,
+        num_kv_heads, max_blocks_per_seq, block_size, num_blocks);
+  else if (head_dim == 64)
+    pa::append_kernel<64><<<(unsigned)grid, threads, 0, st>>>(
+        k, v, kc, vc, block_tables, cu_q_lens, ctx_lens, slot_mapping, num_seqs, num_tokens,
+        num_kv_heads, max_blocks_per_seq, block_size, num_blocks);
+  else
+    return PA_ERR_UNSUPPORTED;
+  return launch_status();
+}
+
 pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs,
                          int num_pairs, int num_kv_heads, int head_dim, int block_size,
                          int num_blocks, pa_dtype dtype, pa_stream_t stream) {

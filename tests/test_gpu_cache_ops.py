@@ -99,3 +99,46 @@ def test_slot_mapping_flags_positions_past_the_table():
     pa.pa_slot_mapping(slots, bt, ctx, w.block_size)
     assert pa.pa_get_device_error() & pa.PA_DEVERR_SEQ_RANGE
     assert int(slots[2]) == -1
+
+
+@pytest.mark.parametrize("factory", [synth.tiny_decode, synth.llama3_8b_gqa_decode])
+def test_fused_append_matches_slot_mapping_plus_scatter(factory):
+    w = factory()
+    kc, vc = to_dev(w.key_cache), to_dev(w.value_cache)
+    slots = torch.full((w.num_seqs,), -7, dtype=torch.int64, device=dev())
+    pa.pa_append(to_dev(w.new_key), to_dev(w.new_value), kc, vc, to_dev(w.block_tables),
+                 to_dev(w.context_lens), slot_mapping=slots)
+    want = oracle_append(w)
+    np.testing.assert_array_equal(slots.cpu().numpy(), want)
+    assert torch.equal(kc.cpu().view(torch.int16), w.key_cache.view(torch.int16))
+    assert torch.equal(vc.cpu().view(torch.int16), w.value_cache.view(torch.int16))
+    assert pa.pa_get_device_error() == 0
+
+
+def test_fused_append_of_prefill_chunks():
+    p = synth.chunked_prefill(seed=5, block_size=32, hq=8, hkv=2, d=128,
+                              ctx_lens=[0, 17, 100, 31], q_lens=[40, 1, 257, 0])
+    kc, vc = to_dev(p.key_cache), to_dev(p.value_cache)
+    pa.pa_append(to_dev(p.new_key), to_dev(p.new_value), kc, vc, to_dev(p.block_tables),
+                 to_dev(p.ctx_lens), cu_q_lens=to_dev(p.cu_q_lens))
+    cuh = p.cu_q_lens.numpy()
+    seq_of = np.repeat(np.arange(p.num_seqs), np.diff(cuh))
+    pos = np.concatenate([np.arange(c, c + n) for c, n in zip(p.ctx_lens.numpy(), np.diff(cuh))])
+    want = oracle.logical_positions_to_slots(p.block_tables.numpy(), seq_of, pos, 32)
+    oracle.reshape_and_cache(int16_view(p.key_cache), int16_view(p.value_cache),
+                             int16_view(p.new_key), int16_view(p.new_value), want, 32)
+    assert torch.equal(kc.cpu().view(torch.int16), p.key_cache.view(torch.int16))
+    assert torch.equal(vc.cpu().view(torch.int16), p.value_cache.view(torch.int16))
+    assert pa.pa_get_device_error() == 0
+
+
+def test_fused_append_flags_positions_past_the_table():
+    w = synth.tiny_decode()
+    kc, vc = to_dev(w.key_cache), to_dev(w.value_cache)
+    ctx = w.context_lens.clone()
+    ctx[1] = w.block_tables.shape[1] * w.block_size
+    slots = torch.zeros(w.num_seqs, dtype=torch.int64, device=dev())
+    pa.pa_append(to_dev(w.new_key), to_dev(w.new_value), kc, vc, to_dev(w.block_tables),
+                 to_dev(ctx), slot_mapping=slots)
+    assert pa.pa_get_device_error() & pa.PA_DEVERR_SEQ_RANGE
+    assert int(slots[1]) == -1
