@@ -81,6 +81,9 @@ struct HalfTiles {
   static constexpr int BOX_BYTES = BS * 128;
   static constexpr int TILE_BYTES = BS * D * 2;
   static constexpr int NS = BS == 16 ? 8 : 4;        // ring depth
+  static constexpr int NW = 4;                       // consumer warps per CTA
+  // resident CTAs per SM to plan registers for, by query n-tiles per CTA
+  static constexpr int min_ctas(int) { return 2; }
   static constexpr int ZERO_CHUNKS_PER_ROW = BOXES * 8;
 
   __device__ static void issue(uint8_t* sk, uint8_t* sv, const CUtensorMap* mk,
@@ -188,7 +191,14 @@ struct E4m3Tiles {
   static constexpr int BOXES = 1;
   static constexpr int BOX_BYTES = BS * 128;
   static constexpr int TILE_BYTES = BS * 128;
-  static constexpr int NS = BS == 16 ? 16 : 8;
+  // Four resident CTAs per SM (96 registers, no meaningful spill) with an
+  // 8-stage ring beat three CTAs with a 16-stage ring by 8% on B200: the FP8
+  // path is latency bound, and more consumer warps per SM hide more of it.
+  // Five or six CTAs per SM force 72 / 64 registers and ~1 KB of spills; so
+  // does four (or three) with two query n-tiles, which therefore plans for two.
+  static constexpr int NS = BS == 16 ? 8 : 4;
+  static constexpr int NW = 4;
+  static constexpr int min_ctas(int nt) { return nt == 1 ? 4 : 2; }
   static constexpr int ZERO_CHUNKS_PER_ROW = 8;
 
   __device__ static void issue(uint8_t* sk, uint8_t* sv, const CUtensorMap* mk,
@@ -328,7 +338,7 @@ __device__ V E4m3Tiles<T, BS>::lds(const uint8_t* tile, int row, int col) {
 template <class Tiles, int BS, int NT>
 struct DecodeShape {
   static constexpr int D = Tiles::D;
-  static constexpr int NW = 4;                      // consumer warps
+  static constexpr int NW = Tiles::NW;              // consumer warps
   static constexpr int THREADS = (NW + 1) * 32;     // + producer warp
   static constexpr int TILE_BYTES = Tiles::TILE_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -343,7 +353,7 @@ struct DecodeShape {
 };
 
 template <class Tiles, int BS, int NT>
-__global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, 2)
+__global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::min_ctas(NT))
     decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
   using Shape = DecodeShape<Tiles, BS, NT>;
