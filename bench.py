@@ -12,8 +12,9 @@ Printed (rank 0, one JSON line): the decode KV bandwidth over the whole step
 the prefill-chunk TFLOP/s of the 8 x 512-token chunk workload, an end-to-end
 figure through the C ABI with host buffers, clocks seen during the timed
 region, the CPU oracle as a baseline, and (single GPU) secondary figures: the
-same decode step over an FP8 pool, copy-on-write block copies and swap
-bandwidth to / from pinned host memory.
+same decode step over an FP8 pool, a mixed batch (decode rows and prefill
+chunks in one launch, against the same work as two calls), copy-on-write
+block copies and swap bandwidth to / from pinned host memory.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 For N > 1 launch with torch.distributed.run; every rank decodes its own batch
@@ -287,6 +288,56 @@ def fp8_decode_measure(dev, steps, warmup, hbm_peak):
             "kv_bytes_per_step": kv}
 
 
+def mixed_measure(dev, steps, warmup):
+    """One chunked-prefill scheduler step: 256 decode rows (GQA decode shape)
+    and 4 prompt chunks of 512 rows over 8192 cached tokens, as one
+    pa_mixed_attention launch and as two calls (pa_decode on the decode rows,
+    then pa_prefill_chunk on the chunks) over the same device buffers."""
+    import paged_kv_cache_397_b200 as pa
+    p = synth.mixed_batch()
+    kc, vc = p.key_cache.to(dev), p.value_cache.to(dev)
+    bt, cl, cu = p.block_tables.to(dev), p.ctx_lens.to(dev), p.cu_q_lens.to(dev)
+    q = p.query.to(dev)
+    pa.pa_append(p.new_key.to(dev), p.new_value.to(dev), kc, vc, bt, cl, cu_q_lens=cu)
+    out = torch.empty_like(q)
+    nd = p.num_decode
+    qlens = torch.diff(p.cu_q_lens)
+    max_q, max_ctx = int(qlens[nd:].max()), int(p.ctx_lens.max())
+    need = max(pa.pa_mixed_workspace_size(nd, p.num_q_heads, p.num_kv_heads, p.head_dim,
+                                          p.block_size, max_ctx),
+               pa.pa_decode_workspace_size(nd, p.num_q_heads, p.num_kv_heads, p.head_dim,
+                                           p.block_size, max_ctx + 1))
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    r0 = int(p.cu_q_lens[nd])
+    d_bt, d_lens = bt[:nd].contiguous(), (cl[:nd] + 1).contiguous()
+    p_bt, p_cl, p_cu = bt[nd:].contiguous(), cl[nd:].contiguous(), (cu[nd:] - r0).contiguous()
+    p_q, p_out, d_out = q[r0:].contiguous(), out[r0:], out[:nd]
+
+    def mixed():
+        pa.pa_mixed_attention(out, q, kc, vc, bt, cu, cl, nd, max_q, max_ctx, p.scale,
+                              workspace=ws)
+
+    def two_calls():
+        pa.pa_decode(d_out, q[:nd], kc, vc, d_bt, d_lens, max_ctx + 1, p.scale, workspace=ws)
+        pa.pa_prefill_chunk(p_out, p_q, kc, vc, p_bt, p_cu, p_cl, max_q, max_ctx, p.scale)
+
+    ms = {"mixed": [], "two": []}
+    for _ in range(2):  # alternate to cancel clock drift
+        for name, fn in (("mixed", mixed), ("two", two_calls)):
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize()
+            ms[name].append(time_steps(fn, steps, torch.cuda.current_stream()) / steps)
+    t_mixed, t_two = min(ms["mixed"]), min(ms["two"])
+    kv = 2 * p.num_kv_heads * p.head_dim * 2 * int((p.ctx_lens[:nd] + 1).sum())
+    flops = 0
+    for c, n in zip(p.ctx_lens[nd:].tolist(), qlens[nd:].tolist()):
+        flops += 4 * p.head_dim * p.num_q_heads * (n * c + n * (n + 1) // 2)
+    return {"workload": p.name, "ms": t_mixed, "ms_two_calls": t_two,
+            "speedup_vs_two_calls": t_two / t_mixed, "decode_kv_bytes": kv,
+            "prefill_causal_flop": flops}
+
+
 def copy_and_swap_measure(dev, steps):
     """Copy-on-write of the shared-prefix workload (128 block pairs) and swap
     of 256 blocks of the GQA decode shape out to pinned host memory and back."""
@@ -518,6 +569,8 @@ def main():
         torch.cuda.empty_cache()
         secondary = {"fp8_decode": fp8_decode_measure(dev, steps=50, warmup=5,
                                                       hbm_peak=hbm_peak)}
+        torch.cuda.empty_cache()
+        secondary["mixed_batch"] = mixed_measure(dev, steps=20, warmup=3)
         torch.cuda.empty_cache()
         secondary.update(copy_and_swap_measure(dev, steps=50))
 

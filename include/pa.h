@@ -312,6 +312,52 @@ pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,
                            int max_blocks_per_seq, float scale, pa_dtype dtype,
                            pa_stream_t stream);
 
+/*
+ * pa_mixed_attention — one launch for a batch that mixes decode rows and
+ * prefill chunks.  "vLLM PagedAttention Deep Dive", "Mechanics of Chunked
+ * Prefill" (the scheduler batches the ongoing decode tokens together with a
+ * chunk of a long prompt, so decode is not starved while the prompt is
+ * processed).
+ * Same rule as pa_prefill_chunk for every sequence: sequence s has
+ * ctx_lens[s] tokens cached before this step and n_s = cu_q_lens[s+1] -
+ * cu_q_lens[s] query rows whose K/V are already written (pa_append with
+ * cu_q_lens) at positions ctx_lens[s] .. ctx_lens[s] + n_s - 1; row i sees
+ * positions 0 .. ctx_lens[s] + i.
+ *   Sequences 0 .. num_decode_seqs - 1 are decode rows: exactly one query
+ *   each, at row s (cu_q_lens[s] == s); a decode row attends over
+ *   ctx_lens[s] + 1 tokens.  Given the same partition_tokens > 0, its result
+ *   is bit-identical to pa_decode with seq_lens = ctx_lens + 1 and
+ *   max_seq_len = max_ctx_len + 1 (with 0, this call picks its own partition
+ *   length: pa_decode's choice capped at 1024 tokens).  A decode sequence
+ *   whose cu_q_lens disagree sets PA_DEVERR_SEQ_RANGE.
+ *   Sequences num_decode_seqs .. num_seqs - 1 are prefill chunks (any length,
+ *   0 included); their rows are bit-identical to pa_prefill_chunk.
+ *   out, query    T[total_q][num_q_heads][head_dim]
+ *   max_q_len     host upper bound on the prefill chunks' lengths
+ *   max_ctx_len   host upper bound on ctx_lens over all sequences;
+ *                 max_ctx_len + 1 <= max_blocks_per_seq * block_size
+ *   workspace     device scratch of at least pa_mixed_workspace_size bytes
+ *                 (0 when there are no decode rows: may then be NULL): the
+ *                 decode rows' work-item queue counter, which this call
+ *                 zeroes on `stream` before its launch, and their split-KV
+ *                 partials.  Calls sharing a workspace must be ordered.
+ * One kernel launch covers both kinds of rows (plus the split-KV combine of
+ * the decode rows when they span several partitions, and the 4-byte memset
+ * of the queue counter).  head_dim must be 128; fp16 / bf16 caches;
+ * group <= 16.
+ */
+pa_status pa_mixed_workspace_size(int num_decode_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int block_size, int max_ctx_len,
+                                  int partition_tokens, size_t *bytes);
+pa_status pa_mixed_attention(void *out, const void *query, const void *key_cache,
+                             const void *value_cache, const int32_t *block_tables,
+                             const int32_t *cu_q_lens, const int32_t *ctx_lens, int num_seqs,
+                             int num_decode_seqs, int total_q, int max_q_len, int max_ctx_len,
+                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                             int num_blocks, int max_blocks_per_seq, int partition_tokens,
+                             float scale, pa_dtype dtype, void *workspace,
+                             size_t workspace_bytes, pa_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Host block manager — the allocator that produces block tables, slot
  * mappings and copy-on-write pairs for the kernels above.  Host memory only;

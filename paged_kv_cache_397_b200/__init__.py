@@ -28,7 +28,8 @@ __all__ = [
     "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
-    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_append", "BlockManager",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_append",
+    "pa_mixed_workspace_size", "pa_mixed_attention", "BlockManager",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
 ]
@@ -62,6 +63,9 @@ _SIGS = {
                            _f, _i, _p, _sz, _p]),
     "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                               _i, _f, _i, _p]),
+    "pa_mixed_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
+    "pa_mixed_attention": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i,
+                                _i, _i, _i, _i, _f, _i, _p, _sz, _p]),
     "pa_get_device_error": (_i, [ctypes.POINTER(ctypes.c_uint), _p]),
     "pa_bm_create": (_i, [_i, _i, _i, ctypes.POINTER(_p)]),
     "pa_bm_destroy": (None, [_p]),
@@ -385,6 +389,49 @@ def pa_prefill_chunk(out, query, key_cache, value_cache, block_tables, cu_q_lens
         S, int(query.shape[0]), int(max_q_len), int(max_ctx_len), int(query.shape[1]), hkv, d,
         bs, nb, int(block_tables.shape[1]), float(scale), _dtype_code(key_cache),
         _stream(stream)))
+    return out
+
+
+def pa_mixed_workspace_size(num_decode_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                            max_ctx_len, partition_tokens=0) -> int:
+    n = ctypes.c_size_t(0)
+    _check("pa_mixed_workspace_size", lib().pa_mixed_workspace_size(
+        int(num_decode_seqs), int(num_q_heads), int(num_kv_heads), int(head_dim),
+        int(block_size), int(max_ctx_len), int(partition_tokens), ctypes.byref(n)))
+    return int(n.value)
+
+
+def pa_mixed_attention(out, query, key_cache, value_cache, block_tables, cu_q_lens, ctx_lens,
+                       num_decode_seqs, max_q_len, max_ctx_len, scale, workspace=None,
+                       partition_tokens=0, stream=None):
+    """Decode rows and prefill chunks in one launch (include/pa.h, pa_mixed_attention).
+
+    The first ``num_decode_seqs`` sequences are decode rows (one query each,
+    at row s); the rest are prefill chunks.  ``workspace`` is a CUDA byte
+    tensor of at least ``pa_mixed_workspace_size`` bytes; allocated with
+    torch when None.
+    """
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [total_q][num_q_heads][head_dim]")
+    if query.dtype != key_cache.dtype or out.dtype != key_cache.dtype:
+        raise ValueError("query/out dtype must match the cache")
+    S, hq = int(ctx_lens.numel()), int(query.shape[1])
+    if cu_q_lens.numel() != S + 1 or block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("cu_q_lens / block_tables do not match ctx_lens")
+    nd = int(num_decode_seqs)
+    need = pa_mixed_workspace_size(nd, hq, hkv, d, bs, int(max_ctx_len), partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_mixed_attention", lib().pa_mixed_attention(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(cu_q_lens, "cu_q_lens", torch.int32, 1), _ptr(ctx_lens, "ctx_lens", torch.int32, 1),
+        S, nd, int(query.shape[0]), int(max_q_len), int(max_ctx_len), hq, hkv, d, bs, nb,
+        int(block_tables.shape[1]), int(partition_tokens), float(scale), _dtype_code(key_cache),
+        ws_ptr, ws_bytes, _stream(stream)))
     return out
 
 

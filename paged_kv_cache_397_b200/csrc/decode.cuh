@@ -61,6 +61,7 @@ struct DecodeParams {
   int max_parts;             // gridDim.x
   float scale_log2;          // softmax scale * log2(e) (FP8: also * k_scale)
   float v_scale;             // FP8: multiplies the output; 1 otherwise
+  int len_add;               // tokens attended = seq_lens[s] + len_add (mixed batch: 1)
 };
 
 // ------------------------------------------------------------------ tiles
@@ -352,189 +353,168 @@ struct DecodeShape {
   static_assert(NS % NW == 0, "ring depth vs consumer warps");
 };
 
-template <class Tiles, int BS, int NT>
-__global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::min_ctas(NT))
-    decode_kernel(const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
-  using Shape = DecodeShape<Tiles, BS, NT>;
-  using T = typename Tiles::Elem;
-  using MmaT = typename Tiles::MmaT;
-  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS;
-  constexpr int GP = NT * 8;  // padded heads per CTA
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Shape::BODY_BYTES);
-  uint64_t* empty_bar = full_bar + NS;
-
-  const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // A length beyond the table or beyond the launch's partitions (max_seq_len)
-  // is a caller error: flag it and attend over the tokens that fit.
-  int L = p.seq_lens[s];
+// Length a work item attends over and its partition count.  A length beyond
+// the table or beyond the launch's partitions (max_seq_len) is a caller error:
+// it is flagged (by the item with flag_errors set) and clamped to what fits.
+template <int BS>
+__device__ __forceinline__ int decode_len(const DecodeParams& p, int s, bool flag_errors) {
+  int L = p.seq_lens[s] + p.len_add;
   const int L_cap = min(p.max_blocks_per_seq, p.max_parts * p.part_blocks) * BS;
   if (L > L_cap) {
-    if (threadIdx.x == 0 && part == 0 && kvh == 0) record_error(PA_DEVERR_SEQ_RANGE);
+    if (flag_errors) record_error(PA_DEVERR_SEQ_RANGE);
     L = L_cap;
   }
-  if (L < 0) L = 0;
-  const int nblk_seq = (L + BS - 1) / BS;
-  const int nparts = nblk_seq == 0 ? 1 : (nblk_seq + p.part_blocks - 1) / p.part_blocks;
-  if (part >= nparts) return;
-  const int blk0 = part * p.part_blocks;
-  const int nblk = min(p.part_blocks, nblk_seq - blk0);  // 0 only when L == 0
+  return L < 0 ? 0 : L;
+}
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
+__device__ __forceinline__ int decode_parts(int nblk_seq, int part_blocks) {
+  return nblk_seq == 0 ? 1 : (nblk_seq + part_blocks - 1) / part_blocks;
+}
+
+// Producer side of one item: issue its nblk (block, KV head) tiles into the
+// ring, ring positions g0 .. g0 + nblk - 1 (position i uses stage i % NS and
+// is that stage's (i / NS)-th fill).  Block ids are fetched once, coalesced.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ bool produce_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                             const DecodeParams& p, uint8_t* ring,
+                                             uint64_t* full_bar, uint64_t* empty_bar, int s,
+                                             int kvh, int blk0, int nblk, int g0, int lane,
+                                             uint64_t policy, bool alive) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  constexpr int NS = Shape::NS;
+  const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+  for (int base = 0; base < nblk; base += 32) {
+    int phys = 0;
+    if (base + lane < nblk) {
+      phys = __ldg(bt + base + lane);
+      if (phys < 0 || phys >= p.num_blocks) {
+        record_error(PA_DEVERR_BLOCK_RANGE);
+        phys = 0;
+      }
     }
-    fence_barrier_init();
+    const int cnt = min(32, nblk - base);
+    for (int j = 0; j < cnt; ++j) {
+      const int ph = __shfl_sync(0xffffffffu, phys, j);
+      if (lane == 0) {
+        const int i = g0 + base + j, st = i % NS;
+        if (i >= NS && alive) alive = mbar_wait(&empty_bar[st], ((i / NS) - 1) & 1);
+        mbar_arrive_expect_tx(&full_bar[st], Shape::STAGE_BYTES);
+        uint8_t* sk = ring + st * Shape::STAGE_BYTES;
+        Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v, (ph * p.num_kv_heads + kvh) * BS,
+                     &full_bar[st], policy);
+      }
+    }
   }
-  __syncthreads();
+  return alive;
+}
 
-  if (warp == NW) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-    }
-    const uint64_t policy = l2_policy_evict_first();
-    const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
-    bool alive = true;
-    for (int base = 0; base < nblk; base += 32) {
-      int phys = 0;
-      if (base + lane < nblk) {
-        phys = __ldg(bt + base + lane);
-        if (phys < 0 || phys >= p.num_blocks) {
-          record_error(PA_DEVERR_BLOCK_RANGE);
-          phys = 0;
-        }
-      }
-      const int cnt = min(32, nblk - base);
-      for (int j = 0; j < cnt; ++j) {
-        const int ph = __shfl_sync(0xffffffffu, phys, j);
-        if (lane == 0) {
-          const int i = base + j, st = i % NS;
-          if (i >= NS && alive) alive = mbar_wait(&empty_bar[st], ((i / NS) - 1) & 1);
-          mbar_arrive_expect_tx(&full_bar[st], Shape::STAGE_BYTES);
-          uint8_t* sk = smem + st * Shape::STAGE_BYTES;
-          Tiles::issue(sk, sk + Shape::TILE_BYTES, &tm_k, &tm_v,
-                       (ph * p.num_kv_heads + kvh) * BS, &full_bar[st], policy);
-        }
-      }
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  const int G = p.group;
-  const int c4 = lane & 3, r4 = lane >> 2;
-  uint32_t qf[D / 16][NT][2];  // Q^T as the B operand
-  Tiles::template load_q<NT>(
-      qf, reinterpret_cast<const T*>(p.query) + ((size_t)s * p.num_q_heads + (size_t)kvh * G) * D,
-      G, lane);
-
-  float m_run[NT][2], l_run[NT][2];
-  float o[D / 16][NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[dt][nt][e] = 0.f;
-  }
-
-  bool alive = true;
-  for (int i = warp; i < nblk; i += NW) {
-    const int st = i % NS;
-    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1);
-    const uint8_t* sk = smem + st * Shape::STAGE_BYTES;
-    const uint8_t* sv = sk + Shape::TILE_BYTES;
-    const int tok_blk = (blk0 + i) * BS;  // logical position of the block's first slot
-    const int valid = min(BS, L - tok_blk);
-    if (valid < BS) {
-      // Slots past the sequence end may hold anything (NaN included); zero
-      // their V rows so that 0-weight x garbage cannot poison the PV product.
-      uint8_t* v_gen = smem + st * Shape::STAGE_BYTES + Shape::TILE_BYTES;
-      constexpr int CPR = Tiles::ZERO_CHUNKS_PER_ROW;
-      for (int idx = lane; idx < (BS - valid) * CPR; idx += 32)
-        *reinterpret_cast<uint4*>(Tiles::zero_chunk(v_gen, valid + idx / CPR, idx % CPR)) =
-            make_uint4(0, 0, 0, 0);
-      __syncwarp();
-    }
-#pragma unroll
-    for (int mt = 0; mt < BS / 16; ++mt) {
-      float sacc[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-      Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
-      // online softmax over this sub-tile's 16 tokens
-      const int t_lo = tok_blk + mt * 16 + r4;
-      const bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
-      // The running max m_run is raised only when a sub-tile's max exceeds
-      // it by more than 8 (log2 units), so P <= 2^8 stays in 16-bit range and
-      // O is rescaled rarely; the stale max cancels in O / l.
-      uint32_t pb[NT][2];
-      float sl[NT][2], sh[NT][2], alpha[NT][2];
-      bool raise = false;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          sl[nt][j] = ok_lo ? sacc[nt][j] * p.scale_log2 : -INFINITY;
-          sh[nt][j] = ok_hi ? sacc[nt][j + 2] * p.scale_log2 : -INFINITY;
-          float mx = fmaxf(sl[nt][j], sh[nt][j]);
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          alpha[nt][j] = 1.f;
-          if (mx > m_run[nt][j] + 8.f) {
-            alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);  // 0 when m_run is -inf
-            m_run[nt][j] = mx;
-            raise = true;
-          }
-        }
-      if (__any_sync(0xffffffffu, raise)) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            l_run[nt][j] *= alpha[nt][j];
-#pragma unroll
-            for (int dt = 0; dt < D / 16; ++dt) {
-              o[dt][nt][j] *= alpha[nt][j];
-              o[dt][nt][j + 2] *= alpha[nt][j];
-            }
-          }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float pv[4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float m_use = m_run[nt][j] == -INFINITY ? 0.f : m_run[nt][j];
-          pv[j] = ex2_approx(sl[nt][j] - m_use);
-          pv[j + 2] = ex2_approx(sh[nt][j] - m_use);
-          l_run[nt][j] += pv[j] + pv[j + 2];
-        }
-        // accumulator rows t / t+8, cols (g, g+1) -> B-operand layout of P^T
-        pb[nt][0] = movmatrix_trans(MmaOp<MmaT>::pack(pv[0], pv[1]));
-        pb[nt][1] = movmatrix_trans(MmaOp<MmaT>::pack(pv[2], pv[3]));
-      }
-      Tiles::template pv<NT>(o, sv, mt, pb, lane);
-    }
-    if (valid < BS) fence_proxy_async_smem();  // our zero stores precede the next TMA write
+// Online softmax of one consumer warp over one (block, KV head) tile whose
+// first slot is logical position tok_blk: S^T = K Q^T, running max and sum,
+// O^T += V^T P^T, on mma.sync with fp32 accumulation.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
+                                              float (&m_run)[NT][2], float (&l_run)[NT][2],
+                                              const uint32_t (&qf)[Tiles::D / 16][NT][2],
+                                              uint8_t* sk, int tok_blk, int L, float scale_log2,
+                                              int lane) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using MmaT = typename Tiles::MmaT;
+  constexpr int D = Shape::D;
+  const int r4 = lane >> 2;
+  uint8_t* sv = sk + Shape::TILE_BYTES;
+  const int valid = min(BS, L - tok_blk);
+  if (valid < BS) {
+    // Slots past the sequence end may hold anything (NaN included); zero
+    // their V rows so that 0-weight x garbage cannot poison the PV product.
+    constexpr int CPR = Tiles::ZERO_CHUNKS_PER_ROW;
+    for (int idx = lane; idx < (BS - valid) * CPR; idx += 32)
+      *reinterpret_cast<uint4*>(Tiles::zero_chunk(sv, valid + idx / CPR, idx % CPR)) =
+          make_uint4(0, 0, 0, 0);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[st]);
   }
+#pragma unroll
+  for (int mt = 0; mt < BS / 16; ++mt) {
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+    Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
+    // online softmax over this sub-tile's 16 tokens
+    const int t_lo = tok_blk + mt * 16 + r4;
+    const bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+    // The running max m_run is raised only when a sub-tile's max exceeds
+    // it by more than 8 (log2 units), so P <= 2^8 stays in 16-bit range and
+    // O is rescaled rarely; the stale max cancels in O / l.
+    uint32_t pb[NT][2];
+    float sl[NT][2], sh[NT][2], alpha[NT][2];
+    bool raise = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        sl[nt][j] = ok_lo ? sacc[nt][j] * scale_log2 : -INFINITY;
+        sh[nt][j] = ok_hi ? sacc[nt][j + 2] * scale_log2 : -INFINITY;
+        float mx = fmaxf(sl[nt][j], sh[nt][j]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        alpha[nt][j] = 1.f;
+        if (mx > m_run[nt][j] + 8.f) {
+          alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);  // 0 when m_run is -inf
+          m_run[nt][j] = mx;
+          raise = true;
+        }
+      }
+    if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          l_run[nt][j] *= alpha[nt][j];
+#pragma unroll
+          for (int dt = 0; dt < D / 16; ++dt) {
+            o[dt][nt][j] *= alpha[nt][j];
+            o[dt][nt][j + 2] *= alpha[nt][j];
+          }
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pv[4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float m_use = m_run[nt][j] == -INFINITY ? 0.f : m_run[nt][j];
+        pv[j] = ex2_approx(sl[nt][j] - m_use);
+        pv[j + 2] = ex2_approx(sh[nt][j] - m_use);
+        l_run[nt][j] += pv[j] + pv[j + 2];
+      }
+      // accumulator rows t / t+8, cols (g, g+1) -> B-operand layout of P^T
+      pb[nt][0] = movmatrix_trans(MmaOp<MmaT>::pack(pv[0], pv[1]));
+      pb[nt][1] = movmatrix_trans(MmaOp<MmaT>::pack(pv[2], pv[3]));
+    }
+    Tiles::template pv<NT>(o, sv, mt, pb, lane);
+  }
+  if (valid < BS) fence_proxy_async_smem();  // our zero stores precede the next TMA write
+}
 
-  // ------------------------------------------------- merge the 4 warp states
+// Merge the NW consumer warps' states of one item in shared memory `mg`
+// ([NW][8 NT][D + 2] floats) in warp order, then write the output row (one
+// partition) or the partition's (m, l, acc) to the workspace.  Opens with a
+// barrier of the consumer warps, so `mg` may alias the item's ring or the
+// previous item's merge area.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void merge_item(float* mg, float (&o)[Tiles::D / 16][NT][4],
+                                           float (&m_run)[NT][2], float (&l_run)[NT][2],
+                                           const DecodeParams& p, int s, int kvh, int part,
+                                           bool single, int ctid, uint32_t bar_consumers) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  constexpr int D = Shape::D, NW = Shape::NW;
+  constexpr int GP = NT * 8;  // padded heads per item
+  const int warp = ctid >> 5, lane = ctid & 31;
+  const int c4 = lane & 3, r4 = lane >> 2;
+  const int G = p.group;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -545,8 +525,7 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::mi
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       l_run[nt][j] = l;
     }
-  named_barrier(1, NW * 32);  // every consumer is done reading the ring
-  float* mg = reinterpret_cast<float*>(smem);  // [NW][GP][D + 2]: acc[D], m, l
+  named_barrier(bar_consumers, NW * 32);  // every consumer is done with `mg`'s old contents
   constexpr int RS = D + 2;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -567,9 +546,8 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::mi
         mg[(warp * GP + g) * RS + D + 1] = l_run[nt][j];
       }
   }
-  named_barrier(1, NW * 32);
-  const bool single = (nparts == 1);
-  for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+  named_barrier(bar_consumers, NW * 32);
+  for (int idx = ctid; idx < G * D; idx += NW * 32) {
     const int g = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
@@ -598,6 +576,99 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::mi
   }
 }
 
+template <class Tiles, int NT>
+__device__ __forceinline__ void reset_state(float (&o)[Tiles::D / 16][NT][4],
+                                            float (&m_run)[NT][2], float (&l_run)[NT][2]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int dt = 0; dt < Tiles::D / 16; ++dt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[dt][nt][e] = 0.f;
+  }
+}
+
+// One work item (split-KV partition `part` of KV head `kvh` of sequence `s`)
+// run by THREADS consecutive threads (`tid` 0 .. THREADS-1) that own the
+// 1024-byte aligned shared memory at `smem` (SMEM_BYTES - 1024 bytes).  They
+// synchronise among themselves only, on named barriers `bar_all` (all
+// THREADS) and `bar_consumers` (the NW consumer warps).
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                            const DecodeParams& p, uint8_t* smem, int part,
+                                            int kvh, int s, int tid, uint32_t bar_all,
+                                            uint32_t bar_consumers) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Shape::BODY_BYTES);
+  uint64_t* empty_bar = full_bar + NS;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  const int L = decode_len<BS>(p, s, tid == 0 && part == 0 && kvh == 0);
+  const int nblk_seq = (L + BS - 1) / BS;
+  const int nparts = decode_parts(nblk_seq, p.part_blocks);
+  if (part >= nparts) return;
+  const int blk0 = part * p.part_blocks;
+  const int nblk = min(p.part_blocks, nblk_seq - blk0);  // 0 only when L == 0
+
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    fence_barrier_init();
+  }
+  named_barrier(bar_all, Shape::THREADS);
+
+  if (warp == NW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(tm_k);
+      tma_prefetch_desc(tm_v);
+    }
+    produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s, kvh, blk0, nblk, 0,
+                                lane, l2_policy_evict_first(), true);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  uint32_t qf[D / 16][NT][2];  // Q^T as the B operand
+  Tiles::template load_q<NT>(
+      qf, reinterpret_cast<const T*>(p.query) +
+              ((size_t)s * p.num_q_heads + (size_t)kvh * p.group) * D,
+      p.group, lane);
+  float m_run[NT][2], l_run[NT][2];
+  float o[D / 16][NT][4];
+  reset_state<Tiles, NT>(o, m_run, l_run);
+  bool alive = true;
+  for (int i = warp; i < nblk; i += NW) {
+    const int st = i % NS;
+    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1);
+    consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
+                                 (blk0 + i) * BS, L, p.scale_log2, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[st]);
+  }
+  // the merge area aliases the ring: merge_item's opening barrier waits for
+  // every consumer to finish reading it
+  merge_item<Tiles, BS, NT>(reinterpret_cast<float*>(smem), o, m_run, l_run, p, s, kvh, part,
+                            nparts == 1, tid, bar_consumers);
+}
+
+template <class Tiles, int BS, int NT>
+__global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::min_ctas(NT))
+    decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  decode_item<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, blockIdx.x, blockIdx.y, blockIdx.z,
+                             threadIdx.x, 0, 1);
+}
+
 // Log-sum-exp combine of split-KV partitions, in partition order.  One CTA
 // of D threads per (sequence, query head); sequences that fit one partition
 // were finished by decode_kernel and are skipped.
@@ -605,7 +676,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(D)
     decode_reduce_kernel(DecodeParams p, int block_size) {
   const int s = blockIdx.x / p.num_q_heads, h = blockIdx.x % p.num_q_heads;
-  int L = p.seq_lens[s];
+  int L = p.seq_lens[s] + p.len_add;
   L = max(0, min(L, min(p.max_blocks_per_seq, p.max_parts * p.part_blocks) * block_size));
   const int nblk = (L + block_size - 1) / block_size;
   const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;

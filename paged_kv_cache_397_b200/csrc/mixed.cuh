@@ -1,0 +1,238 @@
+// mixed.cuh — one launch for a batch that mixes decode rows and prefill chunks.
+//
+// What it computes ("vLLM PagedAttention Deep Dive", "Mechanics of Chunked
+// Prefill": the scheduler puts the ongoing decode tokens and a chunk of a long
+// prompt into the same batch): every query row of the batch attends causally
+// to its own sequence's paged K/V.  Sequence s has ctx_lens[s] tokens cached
+// before this step and cu_q_lens[s+1] - cu_q_lens[s] query rows whose K/V are
+// already in the cache; chunk row i sees positions 0 .. ctx_lens[s] + i.  A
+// decode row is the one-row case: it sees ctx_lens[s] + 1 tokens.
+//
+// How (B200 design).  The first num_decode sequences are decode rows (one
+// query each, at row s); the rest are prefill chunks.  One grid of 384-thread
+// CTAs covers both kinds of work:
+//  * CTAs [0, prefill_ctas) each run one 256-row prefill tile on the tcgen05
+//    tensor cores (prefill_tile, the same code as pa_prefill_chunk), longest
+//    tiles first;
+//  * the remaining CTAs (at most one per SM) each host two persistent decode
+//    workers of 160 threads (a producer warp and four consumer warps, on
+//    their own named barriers and shared memory).  A worker's producer takes
+//    split-KV work items (partition, KV head, decode sequence) from an atomic
+//    queue in the workspace and streams their (block, KV head) tiles through
+//    one TMA ring without draining it between items; the consumers process
+//    each item exactly as pa_decode's CTA does (same warp for each block, same
+//    merge order), so the results are bit-identical to pa_decode.
+// The hardware hands out CTAs in launch order, so the long compute-bound
+// prefill tiles start first; decode workers start on the SMs the prefill tail
+// leaves idle and the queue keeps them all busy until it is drained,
+// whatever the mix of sequence lengths.  Decode items that span several
+// partitions are combined afterwards by decode_reduce_kernel.
+#pragma once
+
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace pa {
+
+// Shared memory of one persistent decode worker: the TMA ring, a merge area
+// of its own (so the producer can stream the next item while the consumers
+// merge this one), ring and item-handoff mbarriers, the item slots, and the
+// item the consumers are working on.
+template <class Tiles, int BS, int NT>
+struct WorkerShape {
+  using Dc = DecodeShape<Tiles, BS, NT>;
+  static constexpr int QD = 2;  // item slots between producer and consumers
+  static constexpr int MERGE_OFF = Dc::RING_BYTES;
+  static constexpr int BAR_OFF = MERGE_OFF + Dc::MERGE_BYTES;
+  static constexpr int NBAR = 2 * Dc::NS + 2 * QD;
+  static constexpr int ITEM_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BYTES = (ITEM_OFF + (QD + 1) * 4 + 1023) / 1024 * 1024;
+};
+
+// A persistent decode worker (THREADS = 160 threads, `tid` 0..159): takes work
+// items i = atomicAdd(queue, 1) until i >= num_items; item i is partition
+// i % max_parts of KV head (i / max_parts) % Hkv of sequence
+// i / (max_parts * Hkv).  Items past a sequence's last partition are skipped
+// by the producer.  Every wait is bounded; a consumer-side timeout ends the
+// worker (and the error word says so).
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              const DecodeParams& p, uint8_t* smem, int* queue,
+                                              int num_items, int tid, uint32_t bar_all,
+                                              uint32_t bar_consumers) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using W = WorkerShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS, QD = W::QD;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + W::BAR_OFF);
+  uint64_t* empty_bar = full_bar + NS;
+  uint64_t* item_full = empty_bar + NS;
+  uint64_t* item_empty = item_full + QD;
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + W::ITEM_OFF);
+  volatile int* cur_item = item_slot + QD;
+  float* mg = reinterpret_cast<float*>(smem + W::MERGE_OFF);
+  const int warp = tid >> 5, lane = tid & 31;
+  const int per_seq = p.max_parts * p.num_kv_heads;
+
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < QD; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_empty[i], 1);
+    }
+    fence_barrier_init();
+  }
+  named_barrier(bar_all, Shape::THREADS);
+
+  if (warp == NW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(tm_k);
+      tma_prefetch_desc(tm_v);
+    }
+    const uint64_t policy = l2_policy_evict_first();
+    bool alive = true;
+    int g = 0;  // ring position of the next tile
+    for (int k = 0;; ++k) {
+      int item = -1, s = 0, kvh = 0, part = 0, nblk = 0;
+      for (;;) {  // next item with work (a bounded scan of the queue)
+        int it = 0;
+        if (lane == 0) it = atomicAdd(queue, 1);
+        it = __shfl_sync(0xffffffffu, it, 0);
+        if (it >= num_items) break;
+        part = it % p.max_parts;
+        kvh = (it / p.max_parts) % p.num_kv_heads;
+        s = it / per_seq;
+        const int L = decode_len<BS>(p, s, lane == 0 && part == 0 && kvh == 0);
+        const int nblk_seq = (L + BS - 1) / BS;
+        if (part < decode_parts(nblk_seq, p.part_blocks)) {
+          item = it;
+          nblk = min(p.part_blocks, nblk_seq - part * p.part_blocks);
+          break;
+        }
+      }
+      const int slot = k % QD;
+      if (lane == 0) {
+        if (k >= QD && alive) alive = mbar_wait(&item_empty[slot], ((k / QD) - 1) & 1);
+        item_slot[slot] = item;
+        mbar_arrive(&item_full[slot]);  // release: the consumers' wait acquires item_slot
+      }
+      if (item < 0) break;
+      alive = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s, kvh,
+                                          part * p.part_blocks, nblk, g, lane, policy, alive);
+      g += nblk;
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  // One thread takes each item from its slot and hands it to all four warps
+  // through cur_item, so the warps always agree on the item (and so reach
+  // the same named barriers) even if a wait times out.
+  int g = 0;
+  for (int k = 0;; ++k) {
+    if (tid == 0) {
+      const int slot = k % QD;
+      const bool ok = mbar_wait(&item_full[slot], (k / QD) & 1);
+      *cur_item = ok ? item_slot[slot] : -1;
+      mbar_arrive(&item_empty[slot]);
+    }
+    __syncwarp();
+    named_barrier(bar_consumers, NW * 32);
+    const int item = *cur_item;
+    if (item < 0) break;
+    const int part = item % p.max_parts;
+    const int kvh = (item / p.max_parts) % p.num_kv_heads;
+    const int s = item / per_seq;
+    const int L = decode_len<BS>(p, s, false);
+    const int nblk_seq = (L + BS - 1) / BS;
+    const int nparts = decode_parts(nblk_seq, p.part_blocks);
+    const int blk0 = part * p.part_blocks;
+    const int nblk = min(p.part_blocks, nblk_seq - blk0);
+    uint32_t qf[D / 16][NT][2];
+    Tiles::template load_q<NT>(
+        qf, reinterpret_cast<const T*>(p.query) +
+                ((size_t)s * p.num_q_heads + (size_t)kvh * p.group) * D,
+        p.group, lane);
+    float m_run[NT][2], l_run[NT][2];
+    float o[D / 16][NT][4];
+    reset_state<Tiles, NT>(o, m_run, l_run);
+    bool alive = true;
+    for (int i = warp; i < nblk; i += NW) {
+      const int gi = g + i, st = gi % NS;
+      if (alive) alive = mbar_wait(&full_bar[st], (gi / NS) & 1);
+      consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
+                                   (blk0 + i) * BS, L, p.scale_log2, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);
+    }
+    g += nblk;
+    // the opening barrier of merge_item also orders this item's read of
+    // cur_item before thread 0 overwrites it for the next item
+    merge_item<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, nparts == 1, tid,
+                              bar_consumers);
+  }
+}
+
+template <typename T, int BS, int NT>
+struct MixedShape {
+  using Pf = PrefillShape<T, BS>;
+  using Tiles = HalfTiles<T, 128, BS>;
+  using Dc = DecodeShape<Tiles, BS, NT>;
+  using Wk = WorkerShape<Tiles, BS, NT>;
+  static constexpr int THREADS = Pf::THREADS;
+  static constexpr int WORKERS = THREADS / Dc::THREADS;  // decode workers per CTA
+  static constexpr int DEC_SMEM = 1024 + WORKERS * Wk::BYTES;
+  static constexpr int SMEM_BYTES = Pf::SMEM_BYTES > DEC_SMEM ? Pf::SMEM_BYTES : DEC_SMEM;
+  static constexpr int MIN_LAUNCH_REGS = Pf::MIN_LAUNCH_REGS;
+  static_assert(WORKERS == 2, "two decode workers per CTA");
+  static_assert(1 + 2 * WORKERS <= 16, "named barrier ids");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+};
+
+struct MixedPlan {
+  int prefill_ctas;       // CTAs [0, prefill_ctas) run prefill tiles
+  int prefill_tiles;      // 256-row tiles per prefill sequence (from max_q_len)
+  int first_prefill_seq;  // == number of decode sequences
+  int decode_items;       // num_decode * num_kv_heads * max_parts
+  int* queue;             // decode work-item counter, zero at launch
+};
+
+template <typename T, int BS, int NT>
+__global__ void __launch_bounds__(MixedShape<T, BS, NT>::THREADS, 1)
+    mixed_kernel(const __grid_constant__ CUtensorMap tm_q,
+                 const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, PrefillParams pp, DecodeParams dp,
+                 MixedPlan plan) {
+  using Sh = MixedShape<T, BS, NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int b = blockIdx.x;
+  if (b < plan.prefill_ctas) {
+    // the last tile of a chunk sees the most keys: hand those out first
+    const int tile = plan.prefill_tiles - 1 - b % plan.prefill_tiles;
+    const int rest = b / plan.prefill_tiles;
+    const int h = rest % pp.num_q_heads;
+    const int s = plan.first_prefill_seq + rest / pp.num_q_heads;
+    prefill_tile<T, BS>(&tm_q, &tm_k, &tm_v, pp, smem, tile, h, s);
+    return;
+  }
+  const int w = threadIdx.x / Sh::Dc::THREADS;
+  if (w >= Sh::WORKERS) return;  // the two spare warps
+  const int tid = threadIdx.x - w * Sh::Dc::THREADS;
+  // decode rows: sequence s must own exactly query row s
+  if (w == 0 && tid == 0) {
+    const int nd = plan.first_prefill_seq;
+    for (int s = b - plan.prefill_ctas; s < nd; s += gridDim.x - plan.prefill_ctas)
+      if (pp.cu_q_lens[s] != s || pp.cu_q_lens[s + 1] != s + 1) record_error(PA_DEVERR_SEQ_RANGE);
+  }
+  decode_worker<typename Sh::Tiles, BS, NT>(&tm_k, &tm_v, dp, smem + w * Sh::Wk::BYTES,
+                                            plan.queue, plan.decode_items, tid, 1 + w,
+                                            1 + Sh::WORKERS + w);
+}
+
+}  // namespace pa

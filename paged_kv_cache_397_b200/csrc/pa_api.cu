@@ -13,6 +13,7 @@
 #include "../../include/pa.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "mixed.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -181,6 +182,80 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   dim3 grid((max_q_len + rows_per_cta - 1) / rows_per_cta, p.num_q_heads, p.num_seqs);
   kern<<<grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return launch_status();
+}
+
+// Split-KV partition length of the decode rows of a mixed batch: as for
+// pa_decode, capped at 1024 tokens so that the decode workers' queue ends in
+// short items (the last item of a worker bounds how long it idles at the end).
+int mixed_partition_tokens(int requested, int num_decode, int num_kv_heads, int block_size,
+                           int max_dec_len) {
+  if (requested > 0) return ((requested + block_size - 1) / block_size) * block_size;
+  const int p = auto_partition_tokens(num_decode, num_kv_heads, block_size, max_dec_len);
+  return p > 1024 ? 1024 : p;
+}
+
+// Bytes of a mixed batch's workspace: 256 of alignment slack, the 256-byte
+// queue-counter block, then the decode rows' split-KV partials.
+size_t mixed_workspace_bytes(int num_decode, int num_q_heads, int head_dim, int num_parts) {
+  if (num_decode <= 0) return 0;
+  size_t b = 512;
+  if (num_parts > 1) b += (size_t)num_decode * num_q_heads * num_parts * (head_dim + 2) * sizeof(float);
+  return b;
+}
+
+int sm_count() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <typename T, int BS, int NT>
+pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const pa::PrefillParams& pp, const pa::DecodeParams& dp,
+                    const pa::MixedPlan& plan, cudaStream_t stream) {
+  using Sh = pa::MixedShape<T, BS, NT>;
+  auto kern = pa::mixed_kernel<T, BS, NT>;
+  static bool configured = false;
+  if (!configured) {
+    // same register-split requirement as prefill_kernel (the prefill tiles
+    // of this kernel run the same setmaxnreg split)
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return PA_ERR_CUDA;
+    if (attr.numRegs < Sh::MIN_LAUNCH_REGS) return PA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Sh::SMEM_BYTES) != cudaSuccess)
+      return PA_ERR_CUDA;
+    configured = true;
+  }
+  // persistent decode workers: at most one CTA (two workers) per SM
+  long long decode_ctas = ((long long)plan.decode_items + Sh::WORKERS - 1) / Sh::WORKERS;
+  if (decode_ctas > sm_count()) decode_ctas = sm_count();
+  const long long grid = plan.prefill_ctas + decode_ctas;
+  if (grid <= 0) return PA_OK;
+  if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
+  kern<<<(unsigned)grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, pp, dp, plan);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (plan.decode_items > 0 && dp.max_parts > 1) {
+    pa::decode_reduce_kernel<T, 128><<<dp.num_seqs * dp.num_q_heads, 128, 0, stream>>>(dp, BS);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+template <typename T, int BS>
+pa_status dispatch_mixed(int group, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const pa::PrefillParams& pp,
+                         const pa::DecodeParams& dp, const pa::MixedPlan& plan,
+                         cudaStream_t stream) {
+  if (group <= 8) return run_mixed<T, BS, 1>(mq, mk, mv, pp, dp, plan, stream);
+  return run_mixed<T, BS, 2>(mq, mk, mv, pp, dp, plan, stream);
 }
 
 }  // namespace
@@ -425,6 +500,7 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
   p.max_parts = num_parts;
   p.scale_log2 = scale * (kv_fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   p.v_scale = kv_fp8 ? v_scale : 1.f;
+  p.len_add = 0;
   auto st = (cudaStream_t)stream;
   if (kv_fp8) {
     if (dtype == PA_BF16) return dispatch_decode_fp8<__nv_bfloat16>(block_size, mk, mv, p, num_parts, st);
@@ -572,6 +648,129 @@ pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
   }
   if (block_size == 16) return run_prefill<__half, 16>(mq, mk, mv, p, max_q_len, st);
   return run_prefill<__half, 32>(mq, mk, mv, p, max_q_len, st);
+}
+
+pa_status pa_mixed_workspace_size(int num_decode_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int block_size, int max_ctx_len,
+                                  int partition_tokens, size_t* bytes) {
+  if (!bytes || num_decode_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_ctx_len < 0 || partition_tokens < 0)
+    return PA_ERR_INVALID_ARG;
+  const int max_dec_len = max_ctx_len + 1;
+  const int pt = mixed_partition_tokens(partition_tokens, num_decode_seqs > 0 ? num_decode_seqs : 1,
+                                        num_kv_heads, block_size, max_dec_len);
+  *bytes = mixed_workspace_bytes(num_decode_seqs, num_q_heads, head_dim,
+                                 (max_dec_len + pt - 1) / pt);
+  return PA_OK;
+}
+
+pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache,
+                             const void* value_cache, const int32_t* block_tables,
+                             const int32_t* cu_q_lens, const int32_t* ctx_lens, int num_seqs,
+                             int num_decode_seqs, int total_q, int max_q_len, int max_ctx_len,
+                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                             int num_blocks, int max_blocks_per_seq, int partition_tokens,
+                             float scale, pa_dtype dtype, void* workspace,
+                             size_t workspace_bytes, pa_stream_t stream) {
+  if (num_seqs < 0 || num_decode_seqs < 0 || num_decode_seqs > num_seqs ||
+      total_q < num_decode_seqs || max_q_len < 0 || max_ctx_len < 0 || num_q_heads <= 0 ||
+      num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0 ||
+      !valid_dtype(dtype) || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || total_q == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !cu_q_lens || !ctx_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  // a decode row attends over ctx + 1 tokens, which must fit the table
+  if ((long long)max_ctx_len >= (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads > 65535) return PA_ERR_INVALID_ARG;
+  if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * num_kv_heads * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
+  if ((long long)total_q * num_q_heads * head_dim > INT_MAX) return PA_ERR_INVALID_ARG;
+
+  // decode rows: split-KV plan over lengths up to max_ctx_len + 1
+  const int num_decode = num_decode_seqs;
+  const int max_dec_len = max_ctx_len + 1;
+  const int pt = mixed_partition_tokens(partition_tokens, num_decode > 0 ? num_decode : 1,
+                                        num_kv_heads, block_size, max_dec_len);
+  const int num_parts = (max_dec_len + pt - 1) / pt;
+  const size_t need = mixed_workspace_bytes(num_decode, num_q_heads, head_dim, num_parts);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return PA_ERR_WORKSPACE;
+  // prefill chunks: 256-row tiles per (chunk, query head)
+  const int num_prefill = num_seqs - num_decode;
+  const long long tiles = (num_prefill > 0 && max_q_len > 0) ? (max_q_len + 255) / 256 : 0;
+  const long long prefill_ctas = tiles * num_q_heads * num_prefill;
+  const long long decode_items = (long long)num_decode * num_kv_heads * num_parts;
+  if (prefill_ctas > INT_MAX || decode_items > INT_MAX) return PA_ERR_INVALID_ARG;
+
+  CUtensorMap mq, mk, mv;
+  const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
+  if (!make_map_2d(&mq, query, (uint64_t)num_q_heads * head_dim, total_q,
+                   (uint64_t)num_q_heads * head_dim, 128, dtype) ||
+      !make_map_2d(&mk, key_cache, head_dim, rows, head_dim, block_size, dtype) ||
+      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, block_size, dtype))
+    return PA_ERR_CUDA;
+
+  pa::PrefillParams pp;
+  pp.out = out;
+  pp.block_tables = block_tables;
+  pp.cu_q_lens = cu_q_lens;
+  pp.ctx_lens = ctx_lens;
+  pp.num_seqs = num_seqs;
+  pp.total_q = total_q;
+  pp.num_q_heads = num_q_heads;
+  pp.num_kv_heads = num_kv_heads;
+  pp.group = group;
+  pp.num_blocks = num_blocks;
+  pp.max_blocks_per_seq = max_blocks_per_seq;
+  pp.scale_log2 = scale * 1.4426950408889634f;
+
+  pa::DecodeParams dp;
+  dp.out = out;
+  dp.query = query;
+  dp.block_tables = block_tables;
+  dp.seq_lens = ctx_lens;
+  dp.len_add = 1;
+  uint8_t* ws_base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
+  float* ws = reinterpret_cast<float*>(ws_base + 256);
+  const size_t acc_elems = (size_t)num_decode * num_q_heads * num_parts * head_dim;
+  dp.ws_acc = num_parts > 1 && need > 0 ? ws : nullptr;
+  dp.ws_ml = num_parts > 1 && need > 0 ? ws + acc_elems : nullptr;
+  dp.num_seqs = num_decode;
+  dp.num_q_heads = num_q_heads;
+  dp.num_kv_heads = num_kv_heads;
+  dp.group = group;
+  dp.num_blocks = num_blocks;
+  dp.max_blocks_per_seq = max_blocks_per_seq;
+  dp.part_blocks = pt / block_size;
+  dp.max_parts = num_parts;
+  dp.scale_log2 = pp.scale_log2;
+  dp.v_scale = 1.f;
+
+  pa::MixedPlan plan;
+  plan.prefill_ctas = (int)prefill_ctas;
+  plan.prefill_tiles = (int)(tiles > 0 ? tiles : 1);
+  plan.first_prefill_seq = num_decode;
+  plan.decode_items = (int)decode_items;
+  plan.queue = need > 0 ? reinterpret_cast<int*>(ws_base) : nullptr;
+
+  auto st = (cudaStream_t)stream;
+  if (plan.queue != nullptr && cudaMemsetAsync(plan.queue, 0, sizeof(int), st) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (dtype == PA_BF16) {
+    if (block_size == 16)
+      return dispatch_mixed<__nv_bfloat16, 16>(group, mq, mk, mv, pp, dp, plan, st);
+    return dispatch_mixed<__nv_bfloat16, 32>(group, mq, mk, mv, pp, dp, plan, st);
+  }
+  if (block_size == 16) return dispatch_mixed<__half, 16>(group, mq, mk, mv, pp, dp, plan, st);
+  return dispatch_mixed<__half, 32>(group, mq, mk, mv, pp, dp, plan, st);
 }
 
 pa_status pa_get_device_error(unsigned int* error_word, pa_stream_t stream) {

@@ -103,17 +103,16 @@ __device__ __forceinline__ void prefill_issue_pv(uint32_t o_tmem, uint32_t p_tme
             (!first || kk > 0) ? 1u : 0u);
 }
 
+// The work of one CTA: chunk rows tile * 256 .. tile * 256 + 255 of query
+// head h of sequence s.  Needs all THREADS threads of the CTA, 1024-byte
+// aligned shared memory at `smem` and all 512 tensor-memory columns.
 template <typename T, int BS>
-__global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+__device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                             const CUtensorMap* tm_v, const PrefillParams& p,
+                                             uint8_t* smem, int tile, int h, int s) {
   using Sh = PrefillShape<T, BS>;
   constexpr int D = Sh::D, BM = Sh::BM, BN = Sh::BN, NQ = Sh::NQ, NS = Sh::NSTAGE;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::BAR_OFF);
   uint64_t* q_full = bars;                        // 1
   uint64_t* ring_full = bars + 1;                 // NS
@@ -123,16 +122,15 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
   uint64_t* o_final = p_full + NQ;                // NQ
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Sh::NBAR);
 
-  const int h = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = p.cu_q_lens[s];
   const int n = p.cu_q_lens[s + 1] - q0;
-  const int i0 = blockIdx.x * (NQ * BM);  // first chunk row of this CTA
+  const int i0 = tile * (NQ * BM);  // first chunk row of this CTA
   if (i0 >= n) return;
   const int c = p.ctx_lens[s];
   int L = c + n;  // tokens in the cache for this sequence
   if (L > p.max_blocks_per_seq * BS) {
-    if (threadIdx.x == 0 && h == 0 && blockIdx.x == 0) record_error(PA_DEVERR_SEQ_RANGE);
+    if (threadIdx.x == 0 && h == 0 && tile == 0) record_error(PA_DEVERR_SEQ_RANGE);
     L = p.max_blocks_per_seq * BS;
   }
   const int kvh = h / p.group;
@@ -171,15 +169,15 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
     const uint64_t pol_kv = l2_policy_evict_last();
     const uint64_t pol_q = l2_policy_evict_first();
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(tm_q);
+      tma_prefetch_desc(tm_k);
+      tma_prefetch_desc(tm_v);
       mbar_arrive_expect_tx(q_full, NQ * Sh::TILE);
     }
     __syncwarp();
     if (lane < 2 * NQ) {  // lane -> (Q tile, 64-column half)
       const int w = lane >> 1, hf = lane & 1;
-      tma_load_2d(smem + Sh::Q_OFF + w * Sh::TILE + hf * Sh::HALF, &tm_q, h * D + hf * 64,
+      tma_load_2d(smem + Sh::Q_OFF + w * Sh::TILE + hf * Sh::HALF, tm_q, h * D + hf * 64,
                   q0 + i0 + w * BM, q_full, pol_q);
     }
     const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq;
@@ -210,7 +208,7 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
         if (lane < 2 * nb) {
           tma_load_2d(smem + Sh::RING_OFF + st * Sh::TILE + (lane & 1) * Sh::HALF +
                           (lane >> 1) * BS * 128,
-                      kv == 0 ? &tm_k : &tm_v, (lane & 1) * 64, row, &ring_full[st], pol_kv);
+                      kv == 0 ? tm_k : tm_v, (lane & 1) * 64, row, &ring_full[st], pol_kv);
         }
       }
     }
@@ -390,6 +388,17 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Sh::TMEM_COLS);
   }
+}
+
+template <typename T, int BS>
+__global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  prefill_tile<T, BS>(&tm_q, &tm_k, &tm_v, p, smem, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 }  // namespace pa

@@ -113,6 +113,7 @@ class PrefillChunkInputs:
     new_value: torch.Tensor
     free_blocks: torch.Tensor
     scale: float
+    num_decode: int = 0  # leading sequences that are decode rows (one query each)
 
     @property
     def num_seqs(self) -> int:
@@ -287,6 +288,37 @@ def chunked_prefill(seed: int = 4, block_size: int = 16, num_seqs: int = 8, ctx:
     gen = torch.Generator().manual_seed(seed)
     ctx_lens = [ctx] * num_seqs if ctx_lens is None else [int(x) for x in ctx_lens]
     q_lens = [chunk] * num_seqs if q_lens is None else [int(x) for x in q_lens]
+    return _chunk_batch(
+        f"chunked_prefill_{len(ctx_lens)}seq_ctx{ctx}_chunk{chunk}_h{hq}kv{hkv}_d{d}_B{block_size}",
+        seed, gen, ctx_lens, q_lens, block_size=block_size, hq=hq, hkv=hkv, d=d, dtype=dtype,
+        pool_factor=pool_factor)
+
+
+def mixed_batch(seed: int = 6, block_size: int = 16, num_decode: int = 256, num_prefill: int = 4,
+                ctx: int = 8192, chunk: int = 512, hq: int = 32, hkv: int = 8, d: int = 128,
+                dtype: torch.dtype = torch.bfloat16, decode_ctx=None, prefill_ctx=None,
+                prefill_q=None, pool_factor: float = 1.25) -> PrefillChunkInputs:
+    """Ongoing decodes and prompt chunks in one batch: ``num_decode`` decode
+    sequences first (one query row each; prior context U[127, 4095], so they
+    attend over 128 .. 4096 tokens like the GQA decode batch), then
+    ``num_prefill`` chunks of ``chunk`` rows against ``ctx`` prior tokens."""
+    gen = torch.Generator().manual_seed(seed)
+    if decode_ctx is None:
+        decode_ctx = torch.randint(127, 4095 + 1, (num_decode,), generator=gen).tolist()
+    decode_ctx = [int(x) for x in decode_ctx]
+    prefill_ctx = [ctx] * num_prefill if prefill_ctx is None else [int(x) for x in prefill_ctx]
+    prefill_q = [chunk] * len(prefill_ctx) if prefill_q is None else [int(x) for x in prefill_q]
+    b = _chunk_batch(
+        f"mixed_batch_{len(decode_ctx)}dec_L128-4096_{len(prefill_ctx)}x{chunk}chunk_ctx{ctx}"
+        f"_h{hq}kv{hkv}_d{d}_B{block_size}",
+        seed, gen, decode_ctx + prefill_ctx, [1] * len(decode_ctx) + prefill_q,
+        block_size=block_size, hq=hq, hkv=hkv, d=d, dtype=dtype, pool_factor=pool_factor)
+    b.num_decode = len(decode_ctx)
+    return b
+
+
+def _chunk_batch(name, seed, gen, ctx_lens, q_lens, *, block_size, hq, hkv, d, dtype,
+                 pool_factor) -> PrefillChunkInputs:
     num_seqs = len(ctx_lens)
     counts = [_ceil_div(c + n, block_size) for c, n in zip(ctx_lens, q_lens)]
     need = sum(counts)
@@ -301,8 +333,7 @@ def chunked_prefill(seed: int = 4, block_size: int = 16, num_seqs: int = 8, ctx:
     cu = torch.zeros(num_seqs + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(torch.tensor(q_lens, dtype=torch.int64), 0).to(torch.int32)
     return PrefillChunkInputs(
-        name=f"chunked_prefill_{num_seqs}seq_ctx{ctx}_chunk{chunk}_h{hq}kv{hkv}_d{d}_B{block_size}",
-        seed=seed, dtype=dtype, block_size=block_size, num_q_heads=hq, num_kv_heads=hkv,
+        name=name, seed=seed, dtype=dtype, block_size=block_size, num_q_heads=hq, num_kv_heads=hkv,
         head_dim=d, num_blocks=num_blocks, ctx_lens=torch.tensor(ctx_lens, dtype=torch.int32),
         cu_q_lens=cu, block_tables=bt, key_cache=kc, value_cache=vc, query=q, new_key=nk,
         new_value=nv, free_blocks=free, scale=1.0 / math.sqrt(d))
@@ -338,6 +369,7 @@ WORKLOADS = {
     "shared_prefix_cow": shared_prefix_cow,
     "long_context_decode": long_context_decode,
     "chunked_prefill": chunked_prefill,
+    "mixed_batch": mixed_batch,
 }
 
 

@@ -73,3 +73,29 @@ def sample_seqs(n_total, k, seed, must=()):
     pick = set(int(x) for x in must)
     pick.update(int(x) for x in rng.choice(n_total, size=min(k, n_total), replace=False))
     return sorted(pick)
+
+
+def oracle_scatter_chunks(p):
+    """Oracle slot mapping + bit scatter of every query row's own K/V of a
+    chunk batch into the CPU caches (in place)."""
+    cu = p.cu_q_lens.numpy()
+    seq_of = np.repeat(np.arange(p.num_seqs), np.diff(cu))
+    pos = np.concatenate([np.arange(c, c + n) for c, n in zip(p.ctx_lens.numpy(), np.diff(cu))])
+    slots = oracle.logical_positions_to_slots(p.block_tables.numpy(), seq_of, pos, p.block_size)
+    oracle.reshape_and_cache(int16_view(p.key_cache), int16_view(p.value_cache),
+                             int16_view(p.new_key), int16_view(p.new_value), slots, p.block_size)
+
+
+def chunk_reference(p, seqs=None, rows=None):
+    """Oracle chunk attention (fp64) for the chosen sequences of a chunk batch,
+    their query rows packed; returns (out, packed cu_q_lens)."""
+    seqs = list(range(p.num_seqs)) if seqs is None else seqs
+    lens = (p.ctx_lens + torch.diff(p.cu_q_lens)).tolist()
+    kc, vc, sbt = sub_pool(p.key_cache, p.value_cache, p.block_tables, lens, seqs, p.block_size)
+    cu = p.cu_q_lens.numpy()
+    qs = [p.query[cu[s]:cu[s + 1]] for s in seqs]
+    sub_cu = np.concatenate([[0], np.cumsum([len(x) for x in qs])])
+    q = torch.cat(qs).double().numpy()
+    ref = oracle.paged_prefill_chunk(q, kc, vc, sbt, sub_cu, [int(p.ctx_lens[s]) for s in seqs],
+                                     p.scale, p.num_kv_heads, rows=rows)
+    return ref, sub_cu

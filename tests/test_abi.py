@@ -61,6 +61,16 @@ def test_workspace_size_is_host_only(lib):
     assert pa.pa_decode_partition_tokens(1, 1, 32, 10) % 32 == 0
     with pytest.raises(pa.PAError):
         pa.pa_decode_workspace_size(4, 0, 4, 64, 16, 65)
+    # mixed batches: no decode rows -> none; decode rows -> the queue counter
+    # block (+ slack), plus partials once they span several partitions
+    assert pa.pa_mixed_workspace_size(0, 8, 2, 128, 16, 100) == 0
+    assert pa.pa_mixed_workspace_size(4, 8, 2, 128, 16, 100, partition_tokens=256) == 512
+    assert pa.pa_mixed_workspace_size(4, 8, 2, 128, 16, 4000, partition_tokens=256) == \
+        512 + 4 * 8 * 16 * (128 + 2) * 4
+    # automatic partitions of a mixed batch are at most 1024 tokens (pa_decode
+    # would take 2048 for this batch)
+    assert pa.pa_decode_partition_tokens(256, 8, 16, 4096) == 2048
+    assert pa.pa_mixed_workspace_size(256, 32, 8, 128, 16, 4095) == 512 + 256 * 32 * 4 * 130 * 4
 
 
 P = ctypes.c_void_p
@@ -107,6 +117,32 @@ def test_prefill_rejects_bad_arguments(lib):
     assert call(d=64) == pa.PA_ERR_UNSUPPORTED
     assert call(bs=64, mb=4) == pa.PA_ERR_UNSUPPORTED
     assert call(tq=0) == pa.PA_OK
+
+
+def test_mixed_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cu=FAKE, cl=FAKE, S=6, nd=4,
+                 tq=68, mq=32, mc=100, hq=8, hkv=2, d=128, bs=16, nb=64, mb=16, pt=0,
+                 scale=0.1, dt=pa.PA_BF16, ws=None, wsb=0, st=None)
+        a.update(kw)
+        return lib.pa_mixed_attention(a["out"], a["q"], a["kc"], a["vc"], a["bt"], a["cu"],
+                                      a["cl"], a["S"], a["nd"], a["tq"], a["mq"], a["mc"],
+                                      a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["mb"],
+                                      a["pt"], a["scale"], a["dt"], a["ws"], a["wsb"], a["st"])
+
+    assert call(nd=7) == pa.PA_ERR_INVALID_ARG                  # more decode rows than seqs
+    assert call(tq=3) == pa.PA_ERR_INVALID_ARG                  # fewer rows than decode seqs
+    assert call(cu=None) == pa.PA_ERR_INVALID_ARG
+    assert call(mc=16 * 16) == pa.PA_ERR_INVALID_ARG            # ctx + 1 does not fit the table
+    assert call(hq=3, hkv=2) == pa.PA_ERR_INVALID_ARG
+    assert call(q=P(0x100004)) == pa.PA_ERR_INVALID_ARG         # misaligned
+    assert call(d=64) == pa.PA_ERR_UNSUPPORTED
+    assert call(hq=34, hkv=2) == pa.PA_ERR_UNSUPPORTED          # group 17
+    assert call(bs=64, mb=4) == pa.PA_ERR_UNSUPPORTED
+    # decode rows long enough to split need a workspace
+    assert call(mc=4000, mb=256, pt=256) == pa.PA_ERR_WORKSPACE
+    assert call(tq=0, nd=0) == pa.PA_OK
+    assert call(S=0, nd=0) == pa.PA_OK
 
 
 def test_cache_ops_reject_bad_arguments(lib):

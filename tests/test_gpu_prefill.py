@@ -6,10 +6,9 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 import paged_kv_cache_397_b200 as pa
 import synth
-from helpers import TOL, dev, int16_view, max_err, sub_pool, to_dev
+from helpers import TOL, chunk_reference, dev, max_err, oracle_scatter_chunks, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -36,27 +35,8 @@ def run_prefill(p):
     return out.cpu()
 
 
-def oracle_scatter(p):
-    cu = p.cu_q_lens.numpy()
-    seq_of = np.repeat(np.arange(p.num_seqs), np.diff(cu))
-    pos = np.concatenate([np.arange(c, c + n) for c, n in zip(p.ctx_lens.numpy(), np.diff(cu))])
-    slots = oracle.logical_positions_to_slots(p.block_tables.numpy(), seq_of, pos, p.block_size)
-    oracle.reshape_and_cache(int16_view(p.key_cache), int16_view(p.value_cache),
-                             int16_view(p.new_key), int16_view(p.new_value), slots, p.block_size)
-
-
-def reference(p, seqs=None, rows=None):
-    seqs = list(range(p.num_seqs)) if seqs is None else seqs
-    lens = (p.ctx_lens + torch.diff(p.cu_q_lens)).tolist()
-    kc, vc, sbt = sub_pool(p.key_cache, p.value_cache, p.block_tables, lens, seqs, p.block_size)
-    cu = p.cu_q_lens.numpy()
-    # queries of the chosen sequences, packed
-    qs = [p.query[cu[s]:cu[s + 1]] for s in seqs]
-    sub_cu = np.concatenate([[0], np.cumsum([len(x) for x in qs])])
-    q = torch.cat(qs).double().numpy()
-    ref = oracle.paged_prefill_chunk(q, kc, vc, sbt, sub_cu, [int(p.ctx_lens[s]) for s in seqs],
-                                     p.scale, p.num_kv_heads, rows=rows)
-    return ref, sub_cu
+oracle_scatter = oracle_scatter_chunks
+reference = chunk_reference
 
 
 @pytest.mark.parametrize("B", [16, 32])

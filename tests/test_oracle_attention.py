@@ -225,6 +225,34 @@ def test_prefill_chunk_equals_masked_sdpa(B):
     del rng
 
 
+def test_mixed_batch_rows_equal_masked_sdpa():
+    # decode rows (one query, ctx + 1 keys) and prefill chunks in one batch:
+    # the chunk rule covers both ("Mechanics of Chunked Prefill")
+    B, hq, hkv, D = 16, 4, 2, 16
+    w = synth.mixed_batch(seed=12, block_size=B, hq=hq, hkv=hkv, d=D, dtype=torch.float16,
+                          decode_ctx=[0, 15, 16, 40], prefill_ctx=[5, 0, 33], prefill_q=[20, 1, 0])
+    assert w.num_decode == 4 and w.cu_q_lens.tolist()[:5] == [0, 1, 2, 3, 4]
+    kc = w.key_cache.double().numpy()
+    vc = w.value_cache.double().numpy()
+    q = w.query.double().numpy()
+    bt = w.block_tables.numpy()
+    cu = w.cu_q_lens.numpy()
+    ctx = w.ctx_lens.numpy()
+    got = oracle.paged_prefill_chunk(q, kc, vc, bt, cu, ctx, w.scale, hkv)
+    for s in range(w.num_seqs):
+        n = int(cu[s + 1] - cu[s])
+        if n == 0:
+            continue
+        L = int(ctx[s]) + n
+        nblk = -(-L // B)
+        K = np.concatenate([kc[bt[s, i]] for i in range(nblk)], axis=1)[:, :L]
+        V = np.concatenate([vc[bt[s, i]] for i in range(nblk)], axis=1)[:, :L]
+        mask = np.arange(L)[None, :] <= (ctx[s] + np.arange(n))[:, None]
+        want = _sdpa(q[cu[s]:cu[s + 1]].transpose(1, 0, 2), K, V, w.scale, mask)
+        np.testing.assert_allclose(got[cu[s]:cu[s + 1]], want.transpose(1, 0, 2), atol=1e-12,
+                                   rtol=0)
+
+
 def test_prefill_row_equals_decode_at_that_length():
     w = synth.chunked_prefill(seed=3, block_size=16, hq=4, hkv=2, d=16, ctx_lens=[21, 0],
                               q_lens=[9, 4], dtype=torch.float16)
