@@ -3,6 +3,7 @@
     python -m paged_kv_cache_397_b200._profile decode  --seqs 32
     python -m paged_kv_cache_397_b200._profile decode-fp8 --seqs 64
     python -m paged_kv_cache_397_b200._profile prefill --seqs 4 [--block-size 16]
+    python -m paged_kv_cache_397_b200._profile mixed --seqs 64
 
 Each case builds a scaled-down copy of a bench workload (same shapes, head
 counts, length distribution and block shuffling; fewer sequences), runs the
@@ -73,9 +74,31 @@ def prefill_case(seqs: int, block_size: int, reps: int = 3):
     print(f"prefill case: {p.name}, causal FLOP per launch {flops}")
 
 
+def mixed_case(seqs: int, reps: int = 3):
+    """`seqs` decode rows (GQA decode lengths) and one 512-row chunk over 8192
+    cached tokens, as one pa_mixed_attention launch."""
+    p = synth.mixed_batch(num_decode=seqs, num_prefill=1)
+    d = torch.device("cuda:0")
+    kc, vc = p.key_cache.to(d), p.value_cache.to(d)
+    bt, cl, cu = p.block_tables.to(d), p.ctx_lens.to(d), p.cu_q_lens.to(d)
+    q = p.query.to(d)
+    pa.pa_append(p.new_key.to(d), p.new_value.to(d), kc, vc, bt, cl, cu_q_lens=cu)
+    out = torch.empty_like(q)
+    nd = p.num_decode
+    qlens = torch.diff(p.cu_q_lens)
+    max_q, max_ctx = int(qlens[nd:].max()), int(p.ctx_lens.max())
+    for _ in range(reps):
+        pa.pa_mixed_attention(out, q, kc, vc, bt, cu, cl, nd, max_q, max_ctx, p.scale)
+    torch.cuda.synchronize()
+    kv = 2 * p.num_kv_heads * p.head_dim * 2 * int((p.ctx_lens[:nd] + 1).sum())
+    flops = sum(4 * p.head_dim * p.num_q_heads * (n * c + n * (n + 1) // 2)
+                for c, n in zip(p.ctx_lens[nd:].tolist(), qlens[nd:].tolist()))
+    print(f"mixed case: {p.name}, decode K/V bytes {kv}, prefill causal FLOP {flops}")
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode", "decode-fp8", "prefill"])
+    ap.add_argument("case", choices=["decode", "decode-fp8", "prefill", "mixed"])
     ap.add_argument("--seqs", type=int, default=None)
     ap.add_argument("--block-size", type=int, default=16)
     a = ap.parse_args()
@@ -84,6 +107,8 @@ def main():
         decode_case(a.seqs or 32)
     elif a.case == "decode-fp8":
         decode_fp8_case(a.seqs or 64)
+    elif a.case == "mixed":
+        mixed_case(a.seqs or 64)
     else:
         prefill_case(a.seqs or 4, a.block_size)
     if pa.pa_get_device_error():
