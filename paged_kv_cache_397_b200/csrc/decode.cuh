@@ -80,6 +80,8 @@ struct HalfTiles {
   static constexpr int D = D_;
   static constexpr int BOXES = D / 64;              // TMA boxes per tile
   static constexpr int BOX_BYTES = BS * 128;
+  static constexpr int HP = 1;                       // KV heads per ring stage
+  static constexpr int TILE_ROWS = BS;               // one cache block per ring stage
   static constexpr int TILE_BYTES = BS * D * 2;
   static constexpr int NS = BS == 16 ? 8 : 4;        // ring depth
   static constexpr int NW = 4;                       // consumer warps per CTA
@@ -87,8 +89,10 @@ struct HalfTiles {
   static constexpr int min_ctas(int) { return 2; }
   static constexpr int ZERO_CHUNKS_PER_ROW = BOXES * 8;
 
+  // K and V of the cache block at pool row `row` into block slot u (always 0)
   __device__ static void issue(uint8_t* sk, uint8_t* sv, const CUtensorMap* mk,
-                               const CUtensorMap* mv, int row, uint64_t* bar, uint64_t pol) {
+                               const CUtensorMap* mv, int row, int /*u*/, uint64_t* bar,
+                               uint64_t pol) {
 #pragma unroll
     for (int h = 0; h < BOXES; ++h) {
       tma_load_2d(sk + h * BOX_BYTES, mk, h * 64, row, bar, pol);
@@ -184,28 +188,39 @@ struct HalfTiles {
 // order d = 16r + 4p + b (r = lane / 4, p = m-tile pair, b = byte), so the
 // V^T fragments of a 16-token sub-tile come from one 16-byte load per token
 // row; byte_perm pairs two token rows along the contraction (token) axis.
-template <typename T, int BS>
+template <typename T, int BS, int HP_ = 1>
 struct E4m3Tiles {
   using Elem = T;
   using MmaT = __half;
   static constexpr int D = 128;
   static constexpr int BOXES = 1;
-  static constexpr int BOX_BYTES = BS * 128;
-  static constexpr int TILE_BYTES = BS * 128;
-  // Four resident CTAs per SM (96 registers, no meaningful spill) with an
-  // 8-stage ring beat three CTAs with a 16-stage ring by 8% on B200: the FP8
-  // path is latency bound, and more consumer warps per SM hide more of it.
-  // Five or six CTAs per SM force 72 / 64 registers and ~1 KB of spills; so
-  // does four (or three) with two query n-tiles, which therefore plans for two.
-  static constexpr int NS = BS == 16 ? 8 : 4;
+  // A ring stage is a 32-row tile of 128-byte rows whatever the cache block
+  // size, and each consumer warp has two stages in flight.  With 16-token
+  // blocks it holds either HP = 2 adjacent KV heads of one block (one
+  // contiguous 4 KB box: the two heads' 2 x G query heads fill the 8-wide MMA
+  // n-tile, each head's columns masked to its own rows) or, when the group
+  // is too wide for that, two blocks of one head (two 2 KB boxes; each starts
+  // on a 1 KB swizzle atom, so the stage reads like one 32-row tile).  On
+  // B200 the FP8 path is latency bound: two 16-row sub-tiles per stage and
+  // two stages per warp (8 stages, 3 CTAs per SM) stream 5.4 TB/s with
+  // 32-token blocks, against 4.6 TB/s for one 16-token block per stage at
+  // four CTAs per SM and 3.5 TB/s for 32-token blocks with 4 stages.
+  static constexpr int HP = HP_;
+  static constexpr int BOX_BYTES = HP * BS * 128;
+  static constexpr int TILE_ROWS = 32;
+  static constexpr int TILE_BYTES = TILE_ROWS * 128;
+  static_assert(HP == 1 || HP * BS == TILE_ROWS, "packed heads fill one stage");
+  static constexpr int NS = 8;
   static constexpr int NW = 4;
-  static constexpr int min_ctas(int nt) { return nt == 1 ? 4 : 2; }
+  static constexpr int min_ctas(int nt) { return nt == 1 ? 3 : 2; }  // two n-tiles: no spill at 2
   static constexpr int ZERO_CHUNKS_PER_ROW = 8;
 
+  // K and V of the cache block at pool row `row` into block slot u of a stage
   __device__ static void issue(uint8_t* sk, uint8_t* sv, const CUtensorMap* mk,
-                               const CUtensorMap* mv, int row, uint64_t* bar, uint64_t pol) {
-    tma_load_2d(sk, mk, 0, row, bar, pol);
-    tma_load_2d(sv, mv, 0, row, bar, pol);
+                               const CUtensorMap* mv, int row, int u, uint64_t* bar,
+                               uint64_t pol) {
+    tma_load_2d(sk + u * BOX_BYTES, mk, 0, row, bar, pol);
+    tma_load_2d(sv + u * BOX_BYTES, mv, 0, row, bar, pol);
   }
   __device__ static uint8_t* zero_chunk(uint8_t* v, int r, int idx) {
     return v + r * 128 + idx * 16;
@@ -243,9 +258,6 @@ struct E4m3Tiles {
       }
     }
   }
-  // Shared-memory tile reads are plain loads through the generic pointer of
-  // the tile (ordered after the stage's barrier wait, free to be scheduled
-  // early against register-only work).
   // Tile reads are volatile shared loads: kept in program order they
   // measured faster here than compiler-scheduled loads.
   template <typename V>
@@ -319,9 +331,9 @@ struct E4m3Tiles {
   }
 };
 
-template <typename T, int BS>
+template <typename T, int BS, int HP_>
 template <typename V>
-__device__ V E4m3Tiles<T, BS>::lds(const uint8_t* tile, int row, int col) {
+__device__ V E4m3Tiles<T, BS, HP_>::lds(const uint8_t* tile, int row, int col) {
   const uint32_t a = sw128(smem_u32(tile), row, col);
   if constexpr (sizeof(V) == 16) {
     V v;
@@ -342,7 +354,12 @@ struct DecodeShape {
   static constexpr int NW = Tiles::NW;              // consumer warps
   static constexpr int THREADS = (NW + 1) * 32;     // + producer warp
   static constexpr int TILE_BYTES = Tiles::TILE_BYTES;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;   // K and V tiles of a stage
+  static constexpr int HP = Tiles::HP;                  // KV heads per stage
+  static constexpr int ROWS = Tiles::TILE_ROWS;         // tile rows per stage
+  static constexpr int TT = ROWS / HP;                  // tokens per stage
+  static constexpr int SB = TT / BS;                    // cache blocks per stage
+  static constexpr int BLOCK_BYTES = STAGE_BYTES / SB;  // K + V bytes of one cache block
   static constexpr int NS = Tiles::NS;              // ring depth
   static constexpr int RING_BYTES = NS * STAGE_BYTES;
   static constexpr int MERGE_BYTES = NW * (NT * 8) * (D + 2) * 4;
@@ -351,6 +368,8 @@ struct DecodeShape {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
   static_assert(NS % NW == 0, "ring depth vs consumer warps");
+  static_assert(TT % BS == 0 && 32 % SB == 0 && ROWS % 16 == 0, "stage vs cache block");
+  static_assert(HP == 1 || SB == 1, "a stage packs heads or blocks, not both");
 };
 
 // Length a work item attends over and its partition count.  A length beyond
@@ -371,9 +390,10 @@ __device__ __forceinline__ int decode_parts(int nblk_seq, int part_blocks) {
   return nblk_seq == 0 ? 1 : (nblk_seq + part_blocks - 1) / part_blocks;
 }
 
-// Producer side of one item: issue its nblk (block, KV head) tiles into the
-// ring, ring positions g0 .. g0 + nblk - 1 (position i uses stage i % NS and
-// is that stage's (i / NS)-th fill).  Block ids are fetched once, coalesced.
+// Producer side of one item: issue its nblk cache blocks, SB per ring stage
+// (the last stage of an item may hold fewer), into ring positions g0, g0 + 1,
+// ... (position i uses stage i % NS and is that stage's (i / NS)-th fill).
+// Block ids are fetched once, coalesced; entries past nblk are never read.
 template <class Tiles, int BS, int NT>
 __device__ __forceinline__ bool produce_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                              const DecodeParams& p, uint8_t* ring,
@@ -381,7 +401,7 @@ __device__ __forceinline__ bool produce_item(const CUtensorMap* tm_k, const CUte
                                              int kvh, int blk0, int nblk, int g0, int lane,
                                              uint64_t policy, bool alive) {
   using Shape = DecodeShape<Tiles, BS, NT>;
-  constexpr int NS = Shape::NS;
+  constexpr int NS = Shape::NS, SB = Shape::SB;
   const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
   for (int base = 0; base < nblk; base += 32) {
     int phys = 0;
@@ -393,56 +413,75 @@ __device__ __forceinline__ bool produce_item(const CUtensorMap* tm_k, const CUte
       }
     }
     const int cnt = min(32, nblk - base);
-    for (int j = 0; j < cnt; ++j) {
-      const int ph = __shfl_sync(0xffffffffu, phys, j);
+    for (int j = 0; j < cnt; j += SB) {
+      int ph[SB];
+#pragma unroll
+      for (int u = 0; u < SB; ++u) ph[u] = __shfl_sync(0xffffffffu, phys, (j + u) & 31);
       if (lane == 0) {
-        const int i = g0 + base + j, st = i % NS;
+        const int nb = min(SB, cnt - j);  // blocks in this stage
+        const int i = g0 + (base + j) / SB, st = i % NS;
         if (i >= NS && alive) alive = mbar_wait(&empty_bar[st], ((i / NS) - 1) & 1);
-        mbar_arrive_expect_tx(&full_bar[st], Shape::STAGE_BYTES);
+        mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
         uint8_t* sk = ring + st * Shape::STAGE_BYTES;
-        Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v, (ph * p.num_kv_heads + kvh) * BS,
-                     &full_bar[st], policy);
+#pragma unroll
+        for (int u = 0; u < SB; ++u)
+          if (u < nb)
+            Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
+                         (ph[u] * p.num_kv_heads + kvh * Shape::HP) * BS, u, &full_bar[st],
+                         policy);
       }
     }
   }
   return alive;
 }
 
-// Online softmax of one consumer warp over one (block, KV head) tile whose
-// first slot is logical position tok_blk: S^T = K Q^T, running max and sum,
-// O^T += V^T P^T, on mma.sync with fp32 accumulation.
+// Online softmax of one consumer warp over one ring stage (TT tokens of HP
+// KV heads) whose first slot is logical position tok_blk: S^T = K Q^T,
+// running max and sum, O^T += V^T P^T, on mma.sync with fp32 accumulation.
+// Positions >= L (the end of the item's tokens) are masked and their V rows
+// zeroed.  With HP > 1, tile rows [h*TT, (h+1)*TT) hold head h of the pack
+// and only query columns [h*G, (h+1)*G) see them.
 template <class Tiles, int BS, int NT>
 __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
                                               float (&m_run)[NT][2], float (&l_run)[NT][2],
                                               const uint32_t (&qf)[Tiles::D / 16][NT][2],
                                               uint8_t* sk, int tok_blk, int L, float scale_log2,
-                                              int lane) {
+                                              int lane, int G = 0) {
   using Shape = DecodeShape<Tiles, BS, NT>;
   using MmaT = typename Tiles::MmaT;
-  constexpr int D = Shape::D;
-  const int r4 = lane >> 2;
+  constexpr int D = Shape::D, TT = Shape::TT, HP = Shape::HP;
+  const int r4 = lane >> 2, c4 = lane & 3;
   uint8_t* sv = sk + Shape::TILE_BYTES;
-  const int valid = min(BS, L - tok_blk);
-  if (valid < BS) {
+  const int valid = min(TT, L - tok_blk);
+  if (valid < TT) {
     // Slots past the sequence end may hold anything (NaN included); zero
     // their V rows so that 0-weight x garbage cannot poison the PV product.
     constexpr int CPR = Tiles::ZERO_CHUNKS_PER_ROW;
-    for (int idx = lane; idx < (BS - valid) * CPR; idx += 32)
-      *reinterpret_cast<uint4*>(Tiles::zero_chunk(sv, valid + idx / CPR, idx % CPR)) =
+    const int per_head = (TT - valid) * CPR;
+    for (int idx = lane; idx < HP * per_head; idx += 32) {
+      const int h = idx / per_head, k = idx % per_head;
+      *reinterpret_cast<uint4*>(Tiles::zero_chunk(sv, h * TT + valid + k / CPR, k % CPR)) =
           make_uint4(0, 0, 0, 0);
+    }
     __syncwarp();
   }
 #pragma unroll
-  for (int mt = 0; mt < BS / 16; ++mt) {
+  for (int mt = 0; mt < Shape::ROWS / 16; ++mt) {
     float sacc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
     Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
-    // online softmax over this sub-tile's 16 tokens
-    const int t_lo = tok_blk + mt * 16 + r4;
-    const bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+    // online softmax over this sub-tile's 16 rows (tokens of one head)
+    const int t_lo = tok_blk + (mt * 16) % TT + r4;
+    bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+    bool col_ok[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        col_ok[nt][j] = HP == 1 || (nt * 8 + 2 * c4 + j) / G == (mt * 16) / TT;
     // The running max m_run is raised only when a sub-tile's max exceeds
     // it by more than 8 (log2 units), so P <= 2^8 stays in 16-bit range and
     // O is rescaled rarely; the stale max cancels in O / l.
@@ -453,8 +492,8 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        sl[nt][j] = ok_lo ? sacc[nt][j] * scale_log2 : -INFINITY;
-        sh[nt][j] = ok_hi ? sacc[nt][j + 2] * scale_log2 : -INFINITY;
+        sl[nt][j] = ok_lo && col_ok[nt][j] ? sacc[nt][j] * scale_log2 : -INFINITY;
+        sh[nt][j] = ok_hi && col_ok[nt][j] ? sacc[nt][j + 2] * scale_log2 : -INFINITY;
         float mx = fmaxf(sl[nt][j], sh[nt][j]);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -495,7 +534,7 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
     }
     Tiles::template pv<NT>(o, sv, mt, pb, lane);
   }
-  if (valid < BS) fence_proxy_async_smem();  // our zero stores precede the next TMA write
+  if (valid < TT) fence_proxy_async_smem();  // our zero stores precede the next TMA write
 }
 
 // Merge the NW consumer warps' states of one item in shared memory `mg`
@@ -514,7 +553,7 @@ __device__ __forceinline__ void merge_item(float* mg, float (&o)[Tiles::D / 16][
   constexpr int GP = NT * 8;  // padded heads per item
   const int warp = ctid >> 5, lane = ctid & 31;
   const int c4 = lane & 3, r4 = lane >> 2;
-  const int G = p.group;
+  const int G = p.group * Shape::HP;  // query heads of the item (kvh is a pack index)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -561,7 +600,7 @@ __device__ __forceinline__ void merge_item(float* mg, float (&o)[Tiles::D / 16][
       den += sc * mg[(w * GP + g) * RS + D + 1];
     }
     num *= p.v_scale;
-    const int h = kvh * G + g;
+    const int h = kvh * G + g;  // == (kvh * HP) * group + g
     if (single) {
       const float v = den > 0.f ? num / den : 0.f;
       reinterpret_cast<T*>(p.out)[((size_t)s * p.num_q_heads + h) * D + d] = T(v);
@@ -636,19 +675,24 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
 
   // -------------------------------------------------------------- consumers
   uint32_t qf[D / 16][NT][2];  // Q^T as the B operand
+  const int G_item = p.group * Shape::HP;  // query heads of this item
   Tiles::template load_q<NT>(
       qf, reinterpret_cast<const T*>(p.query) +
-              ((size_t)s * p.num_q_heads + (size_t)kvh * p.group) * D,
-      p.group, lane);
+              ((size_t)s * p.num_q_heads + (size_t)kvh * G_item) * D,
+      G_item, lane);
   float m_run[NT][2], l_run[NT][2];
   float o[D / 16][NT][4];
   reset_state<Tiles, NT>(o, m_run, l_run);
   bool alive = true;
-  for (int i = warp; i < nblk; i += NW) {
+  const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
+  // a stage may reach past the item's last block (into the next partition)
+  const int L_end = min(L, (blk0 + nblk) * BS);
+  for (int i = warp; i < nstages; i += NW) {
     const int st = i % NS;
     if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1);
     consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
-                                 (blk0 + i) * BS, L, p.scale_log2, lane);
+                                 (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane,
+                                 p.group);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[st]);
   }

@@ -123,7 +123,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
       if (item < 0) break;
       alive = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s, kvh,
                                           part * p.part_blocks, nblk, g, lane, policy, alive);
-      g += nblk;
+      g += (nblk + Shape::SB - 1) / Shape::SB;
     }
     return;
   }
@@ -153,6 +153,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     const int blk0 = part * p.part_blocks;
     const int nblk = min(p.part_blocks, nblk_seq - blk0);
     uint32_t qf[D / 16][NT][2];
+    static_assert(Shape::HP == 1, "the mixed batch's decode workers read one KV head per item");
     Tiles::template load_q<NT>(
         qf, reinterpret_cast<const T*>(p.query) +
                 ((size_t)s * p.num_q_heads + (size_t)kvh * p.group) * D,
@@ -161,15 +162,18 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     float o[D / 16][NT][4];
     reset_state<Tiles, NT>(o, m_run, l_run);
     bool alive = true;
-    for (int i = warp; i < nblk; i += NW) {
+    const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
+    // a stage may reach past the item's last block (into the next partition)
+    const int L_end = min(L, (blk0 + nblk) * BS);
+    for (int i = warp; i < nstages; i += NW) {
       const int gi = g + i, st = gi % NS;
       if (alive) alive = mbar_wait(&full_bar[st], (gi / NS) & 1);
       consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
-                                   (blk0 + i) * BS, L, p.scale_log2, lane);
+                                   (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
-    g += nblk;
+    g += nstages;
     // the opening barrier of merge_item also orders this item's read of
     // cur_item before thread 0 overwrites it for the next item
     merge_item<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, nparts == 1, tid,

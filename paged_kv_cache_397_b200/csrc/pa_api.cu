@@ -122,7 +122,7 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
       return PA_ERR_CUDA;
     configured = true;
   }
-  dim3 grid(num_parts, p.num_kv_heads, p.num_seqs);
+  dim3 grid(num_parts, p.num_kv_heads / Tiles::HP, p.num_seqs);  // y: packs of HP kv heads
   kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (num_parts > 1) {
@@ -151,10 +151,19 @@ pa_status dispatch_decode(int D, int BS, const CUtensorMap& mk, const CUtensorMa
   return PA_ERR_UNSUPPORTED;
 }
 
+// FP8 head packing: with 16-token blocks, two adjacent kv heads share a ring
+// stage (one contiguous 4 KB box) whenever their query heads fit one 8-wide
+// n-tile; the tensor maps' boxes must then be 2 x 16 rows high.
+bool fp8_pack_heads(int block_size, int group, int num_kv_heads) {
+  return block_size == 16 && 2 * group <= 8 && num_kv_heads % 2 == 0;
+}
+
 template <typename T>
 pa_status dispatch_decode_fp8(int BS, const CUtensorMap& mk, const CUtensorMap& mv,
                               pa::DecodeParams p, int num_parts, cudaStream_t stream) {
   using namespace pa;
+  if (BS == 16 && fp8_pack_heads(BS, p.group, p.num_kv_heads))
+    return run_decode<E4m3Tiles<T, 16, 2>, 16, 1>(mk, mv, p, num_parts, stream);
   if (BS == 16) return dispatch_group<E4m3Tiles<T, 16>, 16>(mk, mv, p, num_parts, stream);
   if (BS == 32) return dispatch_group<E4m3Tiles<T, 32>, 32>(mk, mv, p, num_parts, stream);
   return PA_ERR_UNSUPPORTED;
@@ -476,8 +485,12 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
   CUtensorMap mk, mv;
   const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
   const pa_dtype cache_dt = kv_fp8 ? PA_FP8_E4M3 : dtype;
-  if (!make_map_2d(&mk, key_cache, head_dim, rows, head_dim, block_size, cache_dt) ||
-      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, block_size, cache_dt))
+  const uint32_t box_rows =
+      kv_fp8 && fp8_pack_heads(block_size, num_q_heads / num_kv_heads, num_kv_heads)
+          ? 2 * block_size
+          : block_size;
+  if (!make_map_2d(&mk, key_cache, head_dim, rows, head_dim, box_rows, cache_dt) ||
+      !make_map_2d(&mv, value_cache, head_dim, rows, head_dim, box_rows, cache_dt))
     return PA_ERR_CUDA;
 
   pa::DecodeParams p;

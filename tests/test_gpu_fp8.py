@@ -79,7 +79,7 @@ SHAPES = [(torch.bfloat16, 16, 32, 8), (torch.float16, 16, 8, 8), (torch.bfloat1
 
 
 @pytest.mark.parametrize("dtype,B,hq,hkv", SHAPES)
-@pytest.mark.parametrize("partition_tokens", [0, 64])
+@pytest.mark.parametrize("partition_tokens", [0, 48, 64])
 def test_fp8_decode_matches_oracle(dtype, B, hq, hkv, partition_tokens):
     lens = [1, B - 1, B, B + 1, 77, 300, 0, 1030]
     w = synth.random_decode(11 + hq + B, lens, dtype=dtype, block_size=B, hq=hq, hkv=hkv, d=128,
