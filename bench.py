@@ -244,7 +244,9 @@ def prefill_measure(dev, steps, warmup, block_size):
     pa.pa_reshape_and_cache(nk, nv, kc, vc, slots)
     out = torch.empty_like(q)
     qmax, cmax = int(torch.diff(p.cu_q_lens).max()), int(p.ctx_lens.max())
-    fn = lambda: pa.pa_prefill_chunk(out, q, kc, vc, bt, cu, cl, qmax, cmax, p.scale)
+    ws = torch.empty(pa.pa_prefill_workspace_size(p.head_dim), dtype=torch.uint8, device=dev)
+    fn = lambda: pa.pa_prefill_chunk(out, q, kc, vc, bt, cu, cl, qmax, cmax, p.scale,
+                                     workspace=ws)
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -312,6 +314,7 @@ def mixed_measure(dev, steps, warmup):
     d_bt, d_lens = bt[:nd].contiguous(), (cl[:nd] + 1).contiguous()
     p_bt, p_cl, p_cu = bt[nd:].contiguous(), cl[nd:].contiguous(), (cu[nd:] - r0).contiguous()
     p_q, p_out, d_out = q[r0:].contiguous(), out[r0:], out[:nd]
+    pws = torch.empty(pa.pa_prefill_workspace_size(p.head_dim), dtype=torch.uint8, device=dev)
 
     def mixed():
         pa.pa_mixed_attention(out, q, kc, vc, bt, cu, cl, nd, max_q, max_ctx, p.scale,
@@ -319,7 +322,8 @@ def mixed_measure(dev, steps, warmup):
 
     def two_calls():
         pa.pa_decode(d_out, q[:nd], kc, vc, d_bt, d_lens, max_ctx + 1, p.scale, workspace=ws)
-        pa.pa_prefill_chunk(p_out, p_q, kc, vc, p_bt, p_cu, p_cl, max_q, max_ctx, p.scale)
+        pa.pa_prefill_chunk(p_out, p_q, kc, vc, p_bt, p_cu, p_cl, max_q, max_ctx, p.scale,
+                            workspace=pws)
 
     ms = {"mixed": [], "two": []}
     for _ in range(2):  # alternate to cancel clock drift

@@ -302,15 +302,25 @@ pa_status pa_decode_static_workspace(void *out, const void *query, const void *k
  *   cu_q_lens  in   int32[num_seqs + 1], cu_q_lens[num_seqs] == total_q
  *   ctx_lens   in   int32[num_seqs]
  *   max_q_len, max_ctx_len  host upper bounds (size the launch; no sync)
+ *   workspace  device scratch of at least pa_prefill_workspace_size bytes, or
+ *              NULL.  The work is one CTA per 256 chunk rows of a query head
+ *              of a sequence, one CTA per SM at a time; with a workspace, the
+ *              units of the last, partly filled wave are split along the key
+ *              range into 2-4 parts when that shortens the tail, and their
+ *              partial results are combined in part order (deterministic; this call zeroes the
+ *              workspace's counters on `stream` first).  Calls sharing a
+ *              workspace must be ordered.  Without one every unit runs
+ *              whole; the two differ only in fp32 rounding order.
  * head_dim must be 128.
  */
+pa_status pa_prefill_workspace_size(int head_dim, size_t *bytes);
 pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,
                            const void *value_cache, const int32_t *block_tables,
                            const int32_t *cu_q_lens, const int32_t *ctx_lens, int num_seqs,
                            int total_q, int max_q_len, int max_ctx_len, int num_q_heads,
                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                           int max_blocks_per_seq, float scale, pa_dtype dtype,
-                           pa_stream_t stream);
+                           int max_blocks_per_seq, float scale, pa_dtype dtype, void *workspace,
+                           size_t workspace_bytes, pa_stream_t stream);
 
 /*
  * pa_mixed_attention — one launch for a batch that mixes decode rows and
@@ -331,7 +341,8 @@ pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,
  *   length: pa_decode's choice capped at 1024 tokens).  A decode sequence
  *   whose cu_q_lens disagree sets PA_DEVERR_SEQ_RANGE.
  *   Sequences num_decode_seqs .. num_seqs - 1 are prefill chunks (any length,
- *   0 included); their rows are bit-identical to pa_prefill_chunk.
+ *   0 included); their rows are bit-identical to pa_prefill_chunk without a
+ *   workspace (no key-range split).
  *   out, query    T[total_q][num_q_heads][head_dim]
  *   max_q_len     host upper bound on the prefill chunks' lengths
  *   max_ctx_len   host upper bound on ctx_lens over all sequences;

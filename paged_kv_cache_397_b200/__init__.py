@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "PAError", "lib", "lib_path", "EXPORTED_SYMBOLS", "pa_status_string", "pa_version",
     "pa_slot_mapping", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_partition_tokens",
-    "pa_decode_workspace_size", "pa_decode", "pa_decode_static_workspace", "pa_prefill_chunk",
+    "pa_decode_workspace_size", "pa_decode", "pa_decode_static_workspace",
+    "pa_prefill_workspace_size", "pa_prefill_chunk",
     "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
@@ -61,8 +62,9 @@ _SIGS = {
     "pa_swap_blocks": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]),
     "pa_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _f,
                            _f, _i, _p, _sz, _p]),
+    "pa_prefill_workspace_size": (_i, [_i, ctypes.POINTER(_sz)]),
     "pa_prefill_chunk": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i,
-                              _i, _f, _i, _p]),
+                              _i, _f, _i, _p, _sz, _p]),
     "pa_mixed_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "pa_mixed_attention": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i,
                                 _i, _i, _i, _i, _f, _i, _p, _sz, _p]),
@@ -371,9 +373,22 @@ def pa_decode_static_workspace(out, query, key_cache, value_cache, block_tables,
     return out
 
 
+def pa_prefill_workspace_size(head_dim=128) -> int:
+    n = ctypes.c_size_t(0)
+    _check("pa_prefill_workspace_size",
+           lib().pa_prefill_workspace_size(int(head_dim), ctypes.byref(n)))
+    return int(n.value)
+
+
 def pa_prefill_chunk(out, query, key_cache, value_cache, block_tables, cu_q_lens, ctx_lens,
-                     max_q_len, max_ctx_len, scale, stream=None):
-    """Causal chunked-prefill attention against the paged context (include/pa.h)."""
+                     max_q_len, max_ctx_len, scale, workspace=None, split_tail=True,
+                     stream=None):
+    """Causal chunked-prefill attention against the paged context (include/pa.h).
+
+    ``workspace``: a CUDA byte tensor of at least ``pa_prefill_workspace_size``
+    bytes; allocated with torch when None and ``split_tail``.  With
+    ``split_tail=False`` no workspace is passed and no unit is split.
+    """
     nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
     if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
         raise ValueError("query/out must be [total_q][num_q_heads][head_dim]")
@@ -382,13 +397,20 @@ def pa_prefill_chunk(out, query, key_cache, value_cache, block_tables, cu_q_lens
     S = int(ctx_lens.numel())
     if cu_q_lens.numel() != S + 1 or block_tables.dim() != 2 or block_tables.shape[0] != S:
         raise ValueError("cu_q_lens / block_tables do not match ctx_lens")
+    if split_tail and workspace is None:
+        workspace = torch.empty(pa_prefill_workspace_size(d), dtype=torch.uint8,
+                                device=query.device)
+    if not split_tail:
+        workspace = None
+    ws_ptr = _ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("pa_prefill_chunk", lib().pa_prefill_chunk(
         _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
         _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
         _ptr(cu_q_lens, "cu_q_lens", torch.int32, 1), _ptr(ctx_lens, "ctx_lens", torch.int32, 1),
         S, int(query.shape[0]), int(max_q_len), int(max_ctx_len), int(query.shape[1]), hkv, d,
-        bs, nb, int(block_tables.shape[1]), float(scale), _dtype_code(key_cache),
-        _stream(stream)))
+        bs, nb, int(block_tables.shape[1]), float(scale), _dtype_code(key_cache), ws_ptr,
+        ws_bytes, _stream(stream)))
     return out
 
 

@@ -66,8 +66,9 @@ def prefill_case(seqs: int, block_size: int, reps: int = 3):
     q = p.query.to(d)
     out = torch.empty_like(q)
     qmax, cmax = int(torch.diff(p.cu_q_lens).max()), int(p.ctx_lens.max())
+    ws = torch.empty(pa.pa_prefill_workspace_size(p.head_dim), dtype=torch.uint8, device=d)
     for _ in range(reps):
-        pa.pa_prefill_chunk(out, q, kc, vc, bt, cu, cl, qmax, cmax, p.scale)
+        pa.pa_prefill_chunk(out, q, kc, vc, bt, cu, cl, qmax, cmax, p.scale, workspace=ws)
     torch.cuda.synchronize()
     flops = sum(4 * p.head_dim * p.num_q_heads * (n * c + n * (n + 1) // 2)
                 for c, n in zip(p.ctx_lens.tolist(), torch.diff(p.cu_q_lens).tolist()))

@@ -73,6 +73,19 @@ bool valid_cache_dtype(pa_dtype d) { return valid_dtype(d) || d == PA_FP8_E4M3; 
 static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
 
 constexpr int kMaxDevices = 64;
+int sm_count() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 std::mutex g_static_ws_mutex;
 void* g_static_ws_addr[kMaxDevices] = {};
 
@@ -169,6 +182,41 @@ pa_status dispatch_decode_fp8(int BS, const CUtensorMap& mk, const CUtensorMap& 
   return PA_ERR_UNSUPPORTED;
 }
 
+// Workspace of pa_prefill_chunk: 256 bytes of alignment slack, 1 KB of
+// per-unit counters, then the partial rows of up to two waves (2 x #SMs) of
+// split parts: O [parts][256][D] and (m, l) [parts][256][2], fp32.
+constexpr size_t kPrefillCounterBytes = 1024;
+constexpr int kPrefillPartWaves = 2;
+size_t prefill_workspace_bytes(int head_dim) {
+  return 256 + kPrefillCounterBytes +
+         (size_t)kPrefillPartWaves * sm_count() * 256 * (head_dim + 2) * sizeof(float);
+}
+
+// Tail split plan.  Work units (256 rows of a query head of a sequence) run
+// one CTA per SM (the kernel uses all of tensor memory), so `units` take
+// ceil(units / #SMs) waves of about one unit's time each.  The last
+// rem = units mod #SMs units can be cut into k parts along the key range;
+// their rem * k parts then take ceil(rem * k / #SMs) waves of 1/k of a unit.
+// The plan takes the k in 2..4 that minimises that (the smallest on ties),
+// if it beats one whole wave and the parts fit the workspace.
+void plan_prefill_split(pa::PrefillParams& p, long long units, bool have_ws) {
+  const int nsm = sm_count();
+  const long long rem = units % nsm;
+  int best_k = 1;
+  double best_t = 1.0;
+  for (int k = 2; k <= 4 && have_ws && rem > 0; ++k) {
+    if (rem * k > (long long)kPrefillPartWaves * nsm) break;
+    const double t = (double)((rem * k + nsm - 1) / nsm) / k;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best_k = k;
+    }
+  }
+  if (rem > (long long)(kPrefillCounterBytes / sizeof(int))) best_k = 1;
+  p.split = best_k;
+  p.n_full = (int)(best_k > 1 ? units - rem : units);
+}
+
 template <typename T, int BS>
 pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       pa::PrefillParams p, int max_q_len, cudaStream_t stream) {
@@ -187,9 +235,14 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
       return PA_ERR_CUDA;
     configured = true;
   }
-  constexpr int rows_per_cta = Sh::NQ * Sh::BM;
-  dim3 grid((max_q_len + rows_per_cta - 1) / rows_per_cta, p.num_q_heads, p.num_seqs);
-  kern<<<grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  const long long units = (long long)p.tiles_per_seq * p.num_q_heads * p.num_seqs;
+  const long long grid = p.n_full + (units - p.n_full) * p.split;
+  if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
+  if (p.split > 1 &&
+      cudaMemsetAsync(p.counters, 0, (units - p.n_full) * sizeof(int), stream) != cudaSuccess)
+    return PA_ERR_CUDA;
+  kern<<<(unsigned)grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  (void)max_q_len;
   return launch_status();
 }
 
@@ -212,18 +265,6 @@ size_t mixed_workspace_bytes(int num_decode, int num_q_heads, int head_dim, int 
   return b;
 }
 
-int sm_count() {
-  static int cached[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
 
 template <typename T, int BS, int NT>
 pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -609,13 +650,19 @@ pa_status pa_decode_static_workspace(void* out, const void* query, const void* k
                    need > 0 ? (size_t)PA_STATIC_WORKSPACE_BYTES : 0, stream);
 }
 
+pa_status pa_prefill_workspace_size(int head_dim, size_t* bytes) {
+  if (!bytes || head_dim <= 0) return PA_ERR_INVALID_ARG;
+  *bytes = prefill_workspace_bytes(head_dim);
+  return PA_OK;
+}
+
 pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
                            const void* value_cache, const int32_t* block_tables,
                            const int32_t* cu_q_lens, const int32_t* ctx_lens, int num_seqs,
                            int total_q, int max_q_len, int max_ctx_len, int num_q_heads,
                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                           int max_blocks_per_seq, float scale, pa_dtype dtype,
-                           pa_stream_t stream) {
+                           int max_blocks_per_seq, float scale, pa_dtype dtype, void* workspace,
+                           size_t workspace_bytes, pa_stream_t stream) {
   if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || max_ctx_len < 0 || num_q_heads <= 0 ||
       num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || !valid_dtype(dtype) ||
       !std::isfinite(scale))
@@ -654,6 +701,19 @@ pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
   p.num_blocks = num_blocks;
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.tiles_per_seq = (max_q_len + 255) / 256;
+  const bool have_ws = workspace != nullptr && workspace_bytes >= prefill_workspace_bytes(head_dim);
+  plan_prefill_split(p, (long long)p.tiles_per_seq * num_q_heads * num_seqs, have_ws);
+  if (p.split > 1) {
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
+    p.counters = reinterpret_cast<int*>(base);
+    p.ws_o = reinterpret_cast<float*>(base + kPrefillCounterBytes);
+    p.ws_ml = p.ws_o + (size_t)kPrefillPartWaves * sm_count() * 256 * head_dim;
+  } else {
+    p.counters = nullptr;
+    p.ws_o = p.ws_ml = nullptr;
+  }
   auto st = (cudaStream_t)stream;
   if (dtype == PA_BF16) {
     if (block_size == 16) return run_prefill<__nv_bfloat16, 16>(mq, mk, mv, p, max_q_len, st);
@@ -743,6 +803,11 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
   pp.num_blocks = num_blocks;
   pp.max_blocks_per_seq = max_blocks_per_seq;
   pp.scale_log2 = scale * 1.4426950408889634f;
+  pp.tiles_per_seq = (int)(tiles > 0 ? tiles : 1);
+  pp.n_full = (int)prefill_ctas;
+  pp.split = 1;
+  pp.ws_o = pp.ws_ml = nullptr;
+  pp.counters = nullptr;
 
   pa::DecodeParams dp;
   dp.out = out;

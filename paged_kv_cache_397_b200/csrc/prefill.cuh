@@ -48,6 +48,15 @@ struct PrefillParams {
   int num_seqs, total_q, num_q_heads, num_kv_heads, group;
   int num_blocks, max_blocks_per_seq;
   float scale_log2;
+  // Work units (one per 256 chunk rows of a query head of a sequence) in
+  // launch order; units [n_full, ...) are tail units whose KV range is cut
+  // into `split` parts (split == 1: none).
+  int tiles_per_seq;  // 256-row tiles per sequence (from the host's max_q_len)
+  int n_full;
+  int split;
+  float* ws_o;        // [tail parts][D / 4][256] float4: unnormalised O of each part
+  float* ws_ml;       // [tail parts][256][2] (running max in log2 units, sum)
+  int* counters;      // [tail units] parts finished; zero at launch
 };
 
 template <typename T, int BS>
@@ -103,13 +112,85 @@ __device__ __forceinline__ void prefill_issue_pv(uint32_t o_tmem, uint32_t p_tme
             (!first || kk > 0) ? 1u : 0u);
 }
 
+// KV-split tail unit, after this part's partial rows are stored (O as
+// [part][D / 4][256 rows] float4, so a warp's stores and loads are
+// contiguous; (m, l) as [part][256 rows][2]): the 256 softmax threads (row =
+// thread) count the part in; the part that completes the count combines all
+// parts of the unit in part order, so the result does not depend on which
+// part finishes last:
+//   M = max_q m_q,  o = sum_q 2^(m_q - M) O_q / sum_q 2^(m_q - M) l_q.
+template <typename T, int D>
+__device__ __forceinline__ void prefill_combine_tail(const PrefillParams& p, int slot, int row,
+                                                     bool row_valid, T* orow, int* flag) {
+  __threadfence();
+  named_barrier(2, 256);
+  if (threadIdx.x == 0) *flag = atomicAdd(&p.counters[slot], 1) == p.split - 1;
+  named_barrier(2, 256);
+  if (!*flag) return;
+  __threadfence();
+  const size_t base = (size_t)slot * p.split;
+  float mq[4], M = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    mq[q] = q < p.split ? __ldcg(p.ws_ml + ((base + q) * 256 + row) * 2) : -INFINITY;
+    M = fmaxf(M, mq[q]);
+  }
+  const float m_use = M == -INFINITY ? 0.f : M;
+  float sc[4], den = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    sc[q] = q < p.split ? exp2f(mq[q] - m_use) : 0.f;
+    if (q < p.split) den += sc[q] * __ldcg(p.ws_ml + ((base + q) * 256 + row) * 2 + 1);
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  if (!row_valid) return;
+  const float4* ws4 = reinterpret_cast<const float4*>(p.ws_o);
+  constexpr int C = 4;  // float4 per chunk: 16 columns, all parts' loads in flight together
+#pragma unroll 1
+  for (int v0 = 0; v0 < D / 4; v0 += C) {
+    float4 part_rows[4][C];  // the other parts' columns, loaded together
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int c = 0; c < C; ++c)
+        if (q < p.split)
+          part_rows[q][c] = __ldcg(ws4 + ((base + q) * (D / 4) + v0 + c) * 256 + row);
+    float acc[4 * C];
+#pragma unroll
+    for (int e = 0; e < 4 * C; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (q >= p.split) continue;
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const float4 x = part_rows[q][c];
+        acc[4 * c] += sc[q] * x.x;
+        acc[4 * c + 1] += sc[q] * x.y;
+        acc[4 * c + 2] += sc[q] * x.z;
+        acc[4 * c + 3] += sc[q] * x.w;
+      }
+    }
+    uint32_t pk[2 * C];
+#pragma unroll
+    for (int e = 0; e < 2 * C; ++e) pk[e] = MmaOp<T>::pack(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+#pragma unroll
+    for (int c = 0; c < C / 2; ++c)
+      reinterpret_cast<uint4*>(orow + 4 * v0)[c] =
+          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  }
+}
+
 // The work of one CTA: chunk rows tile * 256 .. tile * 256 + 255 of query
-// head h of sequence s.  Needs all THREADS threads of the CTA, 1024-byte
-// aligned shared memory at `smem` and all 512 tensor-memory columns.
+// head h of sequence s, over the whole causal key range (nparts == 1) or over
+// part `part` of it, split into nparts runs of 128-key tiles (tail unit
+// `slot`; the parts' partial rows are combined by the last one to finish).
+// Needs all THREADS threads of the CTA, 1024-byte aligned shared memory at
+// `smem` and all 512 tensor-memory columns.
 template <typename T, int BS>
 __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const PrefillParams& p,
-                                             uint8_t* smem, int tile, int h, int s) {
+                                             uint8_t* smem, int tile, int h, int s, int part = 0,
+                                             int nparts = 1, int slot = 0) {
   using Sh = PrefillShape<T, BS>;
   constexpr int D = Sh::D, BM = Sh::BM, BN = Sh::BN, NQ = Sh::NQ, NS = Sh::NSTAGE;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -121,6 +202,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   uint64_t* p_full = s_full + NQ;                 // NQ
   uint64_t* o_final = p_full + NQ;                // NQ
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Sh::NBAR);
+  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = p.cu_q_lens[s];
@@ -136,8 +218,26 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   const int kvh = h / p.group;
   const int rows = min(NQ * BM, n - i0);            // valid rows of this CTA
   const int kv_end = min(L, c + i0 + rows);         // keys the last valid row needs
-  const int ntiles = (kv_end + BN - 1) / BN;        // >= 1
+  const int ntiles_all = (kv_end + BN - 1) / BN;    // >= 1
+  const int j0 = part * ntiles_all / nparts;         // this part's key tiles [j0, j1)
+  const int ntiles = (part + 1) * ntiles_all / nparts - j0;
   const int nblk_seq = (L + BS - 1) / BS;
+  if (ntiles == 0) {
+    // an empty part of a split unit (fewer key tiles than parts): it counts
+    // in with an empty partial, and may be the one that combines
+    if (warp >= 8) return;
+    const int r = threadIdx.x;  // row of the CTA's 256
+    const size_t u = (size_t)slot * p.split + part;
+    p.ws_ml[(u * 256 + r) * 2] = -INFINITY;
+    p.ws_ml[(u * 256 + r) * 2 + 1] = 0.f;
+    float4* dst = reinterpret_cast<float4*>(p.ws_o) + u * (D / 4) * 256 + r;
+    for (int v = 0; v < D / 4; ++v) dst[v * 256] = make_float4(0.f, 0.f, 0.f, 0.f);
+    prefill_combine_tail<T, D>(p, slot, r, i0 + r < n,
+                               reinterpret_cast<T*>(p.out) +
+                                   ((size_t)(q0 + i0 + r) * p.num_q_heads + h) * D,
+                               last_flag);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -183,7 +283,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq;
     bool alive = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int b0 = j * Sh::BLOCKS_PER_TILE;
+      const int b0 = (j0 + j) * Sh::BLOCKS_PER_TILE;
       const int nb = min(Sh::BLOCKS_PER_TILE, nblk_seq - b0);
       int phys = 0;
       if (lane < nb) {
@@ -276,7 +376,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     for (int j = 0; j < ntiles; ++j) {
       if (alive) alive = mbar_wait(&s_full[w], j & 1);
       tc_fence_after();
-      const int kbase = j * BN;
+      const int kbase = (j0 + j) * BN;
       if (w == 0 && j == ntiles - 1 && L - kbase < BN) {
         // Zero V rows past the sequence end before PV0/PV1 of the last tile.
         // S0_j complete implies every earlier use of V_j's stage landed, so
@@ -333,7 +433,10 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
         m_run = m_tile;
       }
       // P = 2^(S * scale - m): packed FMA, SFU exp2, packed row sums
-      const uint64_t sc2 = f2_pack(sc, sc), negm2 = f2_pack(-m_run, -m_run);
+      // a row with no visible key yet (only in a later part of a split
+      // unit) keeps m_run = -inf: use 0 so that its masked scores give 0
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const uint64_t sc2 = f2_pack(sc, sc), negm2 = f2_pack(-m_use, -m_use);
       uint64_t rsum[4] = {0, 0, 0, 0};  // four packed partial sums
 #pragma unroll
       for (int cc = 0; cc < BN / 16; ++cc) {
@@ -370,16 +473,30 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     tmem_ld32_at<64>(t_o + 64, ov);
     tmem_ld32_at<96>(t_o + 96, ov);
     tmem_wait_ld();
-    if (row < n) {
+    if (nparts == 1) {
+      if (row < n) {
 #pragma unroll
-      for (int v = 0; v < D / 8; ++v) {
-        uint32_t pk[4];
+        for (int v = 0; v < D / 8; ++v) {
+          uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          pk[e] = MmaOp<T>::pack(__uint_as_float(ov[8 * v + 2 * e]) * inv,
-                                 __uint_as_float(ov[8 * v + 2 * e + 1]) * inv);
-        reinterpret_cast<uint4*>(orow)[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          for (int e = 0; e < 4; ++e)
+            pk[e] = MmaOp<T>::pack(__uint_as_float(ov[8 * v + 2 * e]) * inv,
+                                   __uint_as_float(ov[8 * v + 2 * e + 1]) * inv);
+          reinterpret_cast<uint4*>(orow)[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
       }
+    } else {
+      // partial row of this part: unnormalised O, running max, sum
+      const int rr = w * BM + r;  // row of the CTA's 256
+      const size_t u = (size_t)slot * p.split + part;
+      float4* dst = reinterpret_cast<float4*>(p.ws_o) + u * (D / 4) * 256 + rr;
+#pragma unroll
+      for (int v = 0; v < D / 4; ++v)
+        dst[v * 256] = make_float4(__uint_as_float(ov[4 * v]), __uint_as_float(ov[4 * v + 1]),
+                                   __uint_as_float(ov[4 * v + 2]), __uint_as_float(ov[4 * v + 3]));
+      p.ws_ml[(u * 256 + rr) * 2] = m_run;
+      p.ws_ml[(u * 256 + rr) * 2 + 1] = l_run;
+      prefill_combine_tail<T, D>(p, slot, rr, row < n, orow, last_flag);
     }
   }
   tc_fence_before();
@@ -398,7 +515,19 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  prefill_tile<T, BS>(&tm_q, &tm_k, &tm_v, p, smem, blockIdx.x, blockIdx.y, blockIdx.z);
+  // 1-D grid: units in launch order, tail units' parts last
+  const int b = blockIdx.x;
+  int unit = b, part = 0, nparts = 1, slot = 0;
+  if (b >= p.n_full) {
+    slot = (b - p.n_full) / p.split;
+    part = (b - p.n_full) % p.split;
+    nparts = p.split;
+    unit = p.n_full + slot;
+  }
+  const int tile = unit % p.tiles_per_seq;
+  const int h = (unit / p.tiles_per_seq) % p.num_q_heads;
+  const int s = unit / (p.tiles_per_seq * p.num_q_heads);
+  prefill_tile<T, BS>(&tm_q, &tm_k, &tm_v, p, smem, tile, h, s, part, nparts, slot);
 }
 
 }  // namespace pa

@@ -61,6 +61,8 @@ def test_workspace_size_is_host_only(lib):
     assert pa.pa_decode_partition_tokens(1, 1, 32, 10) % 32 == 0
     with pytest.raises(pa.PAError):
         pa.pa_decode_workspace_size(4, 0, 4, 64, 16, 65)
+    # prefill: counters + two waves (148 SMs without a GPU) of 256-row fp32 partials
+    assert pa.pa_prefill_workspace_size(128) == 256 + 1024 + 2 * 148 * 256 * 130 * 4
     # mixed batches: no decode rows -> none; decode rows -> the queue counter
     # block (+ slack), plus partials once they span several partitions
     assert pa.pa_mixed_workspace_size(0, 8, 2, 128, 16, 100) == 0
@@ -104,12 +106,12 @@ def test_prefill_rejects_bad_arguments(lib):
     def call(**kw):
         a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cu=FAKE, cl=FAKE, S=2, tq=64,
                  mq=32, mc=100, hq=8, hkv=2, d=128, bs=16, nb=64, mb=16, scale=0.1,
-                 dt=pa.PA_BF16, st=None)
+                 dt=pa.PA_BF16, ws=None, wsb=0, st=None)
         a.update(kw)
         return lib.pa_prefill_chunk(a["out"], a["q"], a["kc"], a["vc"], a["bt"], a["cu"],
                                     a["cl"], a["S"], a["tq"], a["mq"], a["mc"], a["hq"],
                                     a["hkv"], a["d"], a["bs"], a["nb"], a["mb"], a["scale"],
-                                    a["dt"], a["st"])
+                                    a["dt"], a["ws"], a["wsb"], a["st"])
 
     assert call(cu=None) == pa.PA_ERR_INVALID_ARG
     assert call(mc=16 * 16) == pa.PA_ERR_INVALID_ARG            # context fills the table

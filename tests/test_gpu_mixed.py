@@ -2,8 +2,8 @@
 
 Against the fp64 oracle (the chunk rule of "vLLM PagedAttention Deep Dive",
 "Mechanics of Chunked Prefill", which covers a decode row as a one-row
-chunk), bit-identical to running pa_decode and pa_prefill_chunk separately on
-the two halves of the batch, bit-identical under relabelling of physical
+chunk), bit-identical to running pa_decode and pa_prefill_chunk (without the
+key-range split of its last wave) separately on the two halves of the batch, bit-identical under relabelling of physical
 blocks, and at the full mixed workload (256 decode rows + 4 x 512-row chunks
 over 8192 cached tokens) on sampled rows."""
 import numpy as np
@@ -60,7 +60,7 @@ def run_separately(p, d, partition_tokens=0):
         cu = (d["cu"][nd:] - r0).contiguous()
         pa.pa_prefill_chunk(out[r0:], d["q"][r0:].contiguous(), d["kc"], d["vc"],
                             d["bt"][nd:].contiguous(), cu, d["cl"][nd:].contiguous(),
-                            max(1, _max_q(p)), max_ctx, p.scale)
+                            max(1, _max_q(p)), max_ctx, p.scale, split_tail=False)
     torch.cuda.synchronize()
     return out
 

@@ -20,8 +20,9 @@ def _clean_error_word():
     assert pa.pa_get_device_error() == 0
 
 
-def run_prefill(p):
-    """Slot mapping + scatter of the chunk K/V, then the chunk attention (GPU)."""
+def run_prefill(p, split_tail=True):
+    """Slot mapping + scatter of the chunk K/V, then the chunk attention (GPU);
+    with split_tail the units of the last wave are split along the key range."""
     kc, vc = to_dev(p.key_cache), to_dev(p.value_cache)
     bt, cl, cu = to_dev(p.block_tables), to_dev(p.ctx_lens), to_dev(p.cu_q_lens)
     slots = torch.empty(p.total_q, dtype=torch.int64, device=dev())
@@ -30,7 +31,7 @@ def run_prefill(p):
     out = torch.full(p.query.shape, float("nan"), dtype=p.dtype, device=dev())
     qlens = np.diff(p.cu_q_lens.numpy())
     pa.pa_prefill_chunk(out, to_dev(p.query), kc, vc, bt, cu, cl, int(qlens.max()),
-                        int(p.ctx_lens.max()), p.scale)
+                        int(p.ctx_lens.max()), p.scale, split_tail=split_tail)
     torch.cuda.synchronize()
     return out.cpu()
 
@@ -42,12 +43,15 @@ reference = chunk_reference
 @pytest.mark.parametrize("B", [16, 32])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2)])
-def test_ragged_chunks_match_oracle(B, dtype, hq, hkv):
+@pytest.mark.parametrize("split_tail", [True, False])
+def test_ragged_chunks_match_oracle(B, dtype, hq, hkv, split_tail):
+    # 2 tiles x hq x 5 sequences = 40 or 80 units: with 4 heads the 40 units
+    # are split three ways along the key range, some parts empty (short keys)
     ctx = [0, 5, 40, 200, 129]
     qn = [1, 130, 7, 300, 256]
     p = synth.chunked_prefill(seed=B + hq, block_size=B, hq=hq, hkv=hkv, d=128, dtype=dtype,
                               ctx_lens=ctx, q_lens=qn)
-    out = run_prefill(p)
+    out = run_prefill(p, split_tail)
     oracle_scatter(p)
     ref, _ = reference(p)
     assert max_err(out, ref) <= TOL[dtype]
@@ -75,10 +79,25 @@ def test_full_size_chunked_prefill_sampled_rows(B):
     out = run_prefill(p)
     oracle_scatter(p)
     rows = [0, 1, 63, 127, 128, 200, 255, 256, 383, 384, 510, 511]
-    seqs = [0, 5]
+    seqs = [0, 5, 7]  # 512 units on 148 SMs: the last 68 (sequence 7 and two heads of 6) split
     ref, sub_cu = reference(p, seqs=seqs, rows=rows)
     cu = p.cu_q_lens.numpy()
     got = torch.cat([out[cu[s] + np.array(rows)] for s in seqs])
     want = np.concatenate([ref[sub_cu[i] + np.array(rows)] for i in range(len(seqs))])
     assert max_err(got, want) <= TOL[p.dtype]
     assert torch.isfinite(out.float()).all()
+
+
+def test_split_tail_long_context_matches_oracle():
+    # one sequence, 2 tiles x 8 heads = 16 units, each split four ways over
+    # 8192 + 512 keys (17 key tiles per part on average)
+    p = synth.chunked_prefill(seed=11, block_size=16, num_seqs=1, hq=8, hkv=2)
+    a = run_prefill(p, split_tail=True)
+    b = run_prefill(p, split_tail=False)
+    oracle_scatter(p)
+    rows = [0, 1, 127, 128, 255, 256, 300, 511]
+    ref, _ = reference(p, rows=rows)
+    assert max_err(a[rows], ref[rows]) <= TOL[p.dtype]
+    assert max_err(b[rows], ref[rows]) <= TOL[p.dtype]
+    # the two differ only in fp32 rounding order
+    assert (a.float() - b.float()).abs().max().item() <= TOL[p.dtype]
