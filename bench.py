@@ -162,7 +162,13 @@ def job_throughput(bytes_per_rank_step: int, world: int, steps: int, ms_max: flo
 
 
 class DecodeStep:
-    """Device-resident inputs of one decode step and the C-ABI calls it makes."""
+    """Device-resident inputs of one decode step and the C-ABI calls it makes.
+
+    The per-step inputs (query, new K/V, block tables, context lengths,
+    lengths) live in one staging buffer, each segment 256-byte aligned, so
+    the end-to-end leg moves them with a single host-to-device copy from one
+    pinned host buffer of the same layout; the device tensors are views.
+    """
 
     def __init__(self, w, dev):
         import paged_kv_cache_397_b200 as pa
@@ -171,13 +177,20 @@ class DecodeStep:
         self.dev = dev
         self.kc = w.key_cache.to(dev)
         self.vc = w.value_cache.to(dev)
-        self.bt = w.block_tables.to(dev)
-        self.ctx = w.context_lens.to(dev)
-        self.lens = (w.context_lens + 1).to(dev)
-        self.q = w.query.to(dev)
-        self.nk = w.new_key.to(dev)
-        self.nv = w.new_value.to(dev)
-        self.slots = torch.empty(w.num_seqs, dtype=torch.int64, device=dev)
+        inputs = [w.query, w.new_key, w.new_value, w.block_tables, w.context_lens,
+                  (w.context_lens + 1).to(torch.int32)]
+        offs, total = [], 0
+        for t in inputs:
+            offs.append(total)
+            total += -(-t.numel() * t.element_size() // 256) * 256
+        self.h_stage = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        for t, o in zip(inputs, offs):
+            n = t.numel() * t.element_size()
+            self.h_stage[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+        self.d_stage = self.h_stage.to(dev)
+        views = [self.d_stage[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                 for t, o in zip(inputs, offs)]
+        self.q, self.nk, self.nv, self.bt, self.ctx, self.lens = views
         self.out = torch.empty_like(self.q)
         self.max_len = int(w.context_lens.max()) + 1
         need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads,
@@ -186,18 +199,10 @@ class DecodeStep:
         self.num_parts = math.ceil(self.max_len / pa.pa_decode_partition_tokens(
             w.num_seqs, w.num_kv_heads, w.block_size, self.max_len))
         self.launches_per_step = 2 + (1 if self.num_parts > 1 else 0)
-        total = int(self.lens.sum())
-        self.kv_bytes = 2 * w.num_kv_heads * w.head_dim * 2 * total  # K and V, bf16
-        # host-side copies for the end-to-end leg (pinned)
-        self.h_q = w.query.pin_memory()
-        self.h_nk = w.new_key.pin_memory()
-        self.h_nv = w.new_value.pin_memory()
-        self.h_bt = w.block_tables.pin_memory()
-        self.h_ctx = w.context_lens.pin_memory()
-        self.h_lens = (w.context_lens + 1).pin_memory()
+        total_tokens = int(self.lens.sum())
+        self.kv_bytes = 2 * w.num_kv_heads * w.head_dim * 2 * total_tokens  # K and V, bf16
         self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
-        self.h2d_bytes = sum(t.numel() * t.element_size() for t in
-                             (self.h_q, self.h_nk, self.h_nv, self.h_bt, self.h_ctx, self.h_lens))
+        self.h2d_bytes = total  # the whole staging buffer (inputs + alignment padding)
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
 
     def append(self):
@@ -213,9 +218,7 @@ class DecodeStep:
         self.decode()
 
     def step_e2e(self):
-        for h, d in ((self.h_q, self.q), (self.h_nk, self.nk), (self.h_nv, self.nv),
-                     (self.h_bt, self.bt), (self.h_ctx, self.ctx), (self.h_lens, self.lens)):
-            d.copy_(h, non_blocking=True)
+        self.d_stage.copy_(self.h_stage, non_blocking=True)
         self.step()
         self.h_out.copy_(self.out, non_blocking=True)
 
