@@ -713,31 +713,55 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::mi
                              threadIdx.x, 0, 1);
 }
 
-// Log-sum-exp combine of split-KV partitions, in partition order.  One CTA
-// of D threads per (sequence, query head); sequences that fit one partition
-// were finished by decode_kernel and are skipped.
+// Log-sum-exp combine of split-KV partitions, in partition order.  One warp
+// per (sequence, query head), REDUCE_WARPS warps per CTA, so the whole grid
+// is one wave of short-lived warps; lane l owns D / 32 consecutive head-dim
+// elements (one vector load per partition).  Per element the arithmetic is
+// M = max_q m_q, num = sum_q 2^(m_q - M) acc_q, den = sum_q 2^(m_q - M) l_q
+// in partition order.  Sequences that fit one partition were finished by
+// decode_kernel and are skipped.
+constexpr int REDUCE_WARPS = 8;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(REDUCE_WARPS * 32)
     decode_reduce_kernel(DecodeParams p, int block_size) {
-  const int s = blockIdx.x / p.num_q_heads, h = blockIdx.x % p.num_q_heads;
+  constexpr int VPL = D / 32;  // elements per lane: 4 (D = 128) or 2 (D = 64)
+  const int lane = threadIdx.x & 31;
+  const int unit = blockIdx.x * REDUCE_WARPS + (threadIdx.x >> 5);
+  if (unit >= p.num_seqs * p.num_q_heads) return;
+  const int s = unit / p.num_q_heads, h = unit % p.num_q_heads;
   int L = p.seq_lens[s] + p.len_add;
   L = max(0, min(L, min(p.max_blocks_per_seq, p.max_parts * p.part_blocks) * block_size));
   const int nblk = (L + block_size - 1) / block_size;
   const int nparts = nblk == 0 ? 1 : (nblk + p.part_blocks - 1) / p.part_blocks;
   if (nparts <= 1) return;
   const size_t row0 = ((size_t)s * p.num_q_heads + h) * p.max_parts;
-  const int d = threadIdx.x;
   float M = -INFINITY;
-  for (int q = 0; q < nparts; ++q) M = fmaxf(M, p.ws_ml[(row0 + q) * 2]);
+#pragma unroll 4
+  for (int q = 0; q < nparts; ++q) M = fmaxf(M, __ldg(p.ws_ml + (row0 + q) * 2));
   const float m_use = M == -INFINITY ? 0.f : M;
-  float num = 0.f, den = 0.f;
+  float num[VPL], den = 0.f;
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) num[e] = 0.f;
+#pragma unroll 4
   for (int q = 0; q < nparts; ++q) {
-    const float sc = exp2f(p.ws_ml[(row0 + q) * 2] - m_use);
-    num += sc * p.ws_acc[(row0 + q) * D + d];
-    den += sc * p.ws_ml[(row0 + q) * 2 + 1];
+    const float sc = exp2f(__ldg(p.ws_ml + (row0 + q) * 2) - m_use);
+    const float* acc = p.ws_acc + (row0 + q) * D + lane * VPL;
+    float a[VPL];
+    if constexpr (VPL == 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(acc));
+      a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+    } else {
+      const float2 v = __ldg(reinterpret_cast<const float2*>(acc));
+      a[0] = v.x; a[1] = v.y;
+    }
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) num[e] += sc * a[e];
+    den += sc * __ldg(p.ws_ml + (row0 + q) * 2 + 1);
   }
-  const float v = den > 0.f ? num / den : 0.f;
-  reinterpret_cast<T*>(p.out)[((size_t)s * p.num_q_heads + h) * D + d] = T(v);
+  T* o = reinterpret_cast<T*>(p.out) + ((size_t)s * p.num_q_heads + h) * D + lane * VPL;
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) o[e] = T(den > 0.f ? num[e] / den : 0.f);
 }
 
 }  // namespace pa

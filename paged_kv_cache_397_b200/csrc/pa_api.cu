@@ -139,8 +139,10 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
   kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (num_parts > 1) {
-    pa::decode_reduce_kernel<T, Shape::D><<<p.num_seqs * p.num_q_heads, Shape::D, 0, stream>>>(
-        p, BS);
+    const int units = p.num_seqs * p.num_q_heads;
+    pa::decode_reduce_kernel<T, Shape::D>
+        <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
+            p, BS);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
@@ -293,7 +295,10 @@ pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   kern<<<(unsigned)grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, pp, dp, plan);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (plan.decode_items > 0 && dp.max_parts > 1) {
-    pa::decode_reduce_kernel<T, 128><<<dp.num_seqs * dp.num_q_heads, 128, 0, stream>>>(dp, BS);
+    const int units = dp.num_seqs * dp.num_q_heads;
+    pa::decode_reduce_kernel<T, 128>
+        <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
+            dp, BS);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
