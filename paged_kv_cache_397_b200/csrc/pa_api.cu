@@ -221,7 +221,7 @@ void plan_prefill_split(pa::PrefillParams& p, long long units, bool have_ws) {
 
 template <typename T, int BS>
 pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      pa::PrefillParams p, int max_q_len, cudaStream_t stream) {
+                      pa::PrefillParams p, cudaStream_t stream) {
   using Sh = pa::PrefillShape<T, BS>;
   auto kern = pa::prefill_kernel<T, BS>;
   static bool configured = false;
@@ -244,7 +244,6 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
       cudaMemsetAsync(p.counters, 0, (units - p.n_full) * sizeof(int), stream) != cudaSuccess)
     return PA_ERR_CUDA;
   kern<<<(unsigned)grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
-  (void)max_q_len;
   return launch_status();
 }
 
@@ -721,11 +720,11 @@ pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
   }
   auto st = (cudaStream_t)stream;
   if (dtype == PA_BF16) {
-    if (block_size == 16) return run_prefill<__nv_bfloat16, 16>(mq, mk, mv, p, max_q_len, st);
-    return run_prefill<__nv_bfloat16, 32>(mq, mk, mv, p, max_q_len, st);
+    if (block_size == 16) return run_prefill<__nv_bfloat16, 16>(mq, mk, mv, p, st);
+    return run_prefill<__nv_bfloat16, 32>(mq, mk, mv, p, st);
   }
-  if (block_size == 16) return run_prefill<__half, 16>(mq, mk, mv, p, max_q_len, st);
-  return run_prefill<__half, 32>(mq, mk, mv, p, max_q_len, st);
+  if (block_size == 16) return run_prefill<__half, 16>(mq, mk, mv, p, st);
+  return run_prefill<__half, 32>(mq, mk, mv, p, st);
 }
 
 pa_status pa_mixed_workspace_size(int num_decode_seqs, int num_q_heads, int num_kv_heads,
