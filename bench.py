@@ -3,12 +3,12 @@
 One step = one decode iteration of the Llama-3-8B-shaped GQA batch (256
 sequences, 32 q / 8 kv heads, head_dim 128, bf16, 16-token blocks, lengths
 uniform in [128, 4096], shuffled physical blocks): slot mapping of the new
-token of every sequence and the scatter of its K/V (one fused launch,
-pa_append), split-KV paged decode and the log-sum-exp reduce — all through
+token of every sequence, the scatter of its K/V and split-KV paged decode in
+one launch (pa_append_decode), then the log-sum-exp combine — all through
 libpa.so's C ABI.
 
 Printed (rank 0, one JSON line): the decode KV bandwidth over the whole step
-(GB/s of algorithmic K/V bytes), decode tokens/s, the roofline of pa_decode,
+(GB/s of algorithmic K/V bytes), decode tokens/s, the roofline of the decode launch,
 the prefill-chunk TFLOP/s of the 8 x 512-token chunk workload, an end-to-end
 figure through the C ABI with host buffers, clocks seen during the timed
 region, the CPU oracle as a baseline, and (single GPU) secondary figures: the
@@ -198,24 +198,18 @@ class DecodeStep:
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
         self.num_parts = math.ceil(self.max_len / pa.pa_decode_partition_tokens(
             w.num_seqs, w.num_kv_heads, w.block_size, self.max_len))
-        self.launches_per_step = 2 + (1 if self.num_parts > 1 else 0)
+        self.launches_per_step = 1 + (1 if self.num_parts > 1 else 0)  # decode + combine
         total_tokens = int(self.lens.sum())
         self.kv_bytes = 2 * w.num_kv_heads * w.head_dim * 2 * total_tokens  # K and V, bf16
         self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         self.h2d_bytes = total  # the whole staging buffer (inputs + alignment padding)
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
 
-    def append(self):
-        # slot mapping + scatter of the new token, fused in one launch
-        self.pa.pa_append(self.nk, self.nv, self.kc, self.vc, self.bt, self.ctx)
-
-    def decode(self):
-        self.pa.pa_decode(self.out, self.q, self.kc, self.vc, self.bt, self.lens, self.max_len,
-                          self.w.scale, workspace=self.ws)
-
     def step(self):
-        self.append()
-        self.decode()
+        # slot of each new token, scatter of its K/V, split-KV decode over the
+        # grown sequences: one decode launch (+ the split-KV combine)
+        self.pa.pa_append_decode(self.out, self.q, self.nk, self.nv, self.kc, self.vc, self.bt,
+                                 self.ctx, self.max_len - 1, self.w.scale, workspace=self.ws)
 
     def step_e2e(self):
         self.d_stage.copy_(self.h_stage, non_blocking=True)
@@ -529,9 +523,8 @@ def main():
     t_stop = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        st.append()
         ev[i][0].record(stream)
-        st.decode()
+        st.step()
         ev[i][1].record(stream)
     t_stop.record(stream)
     torch.cuda.synchronize()
@@ -596,7 +589,8 @@ def main():
                        "parallelism": f"replicas x{world} (each rank its own batch)"},
             "hbm_frac": value / world / hbm_peak,
             "decode_tokens_per_s": world * w.num_seqs / (ms_step * 1e-3),
-            "roofline": {"kernel": "pa_decode (decode_kernel + decode_reduce_kernel)",
+            "roofline": {"kernel": "pa_append_decode (decode_kernel with the fused append + "
+                                   "decode_reduce_kernel)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
                          "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
                          "peak_kind": f"hbm copy, {peak_kind}"},

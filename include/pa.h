@@ -236,6 +236,35 @@ pa_status pa_decode(void *out, const void *query, const void *key_cache, const v
                     size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_append_decode — one decode step in one launch: pa_append of every
+ * sequence's new token followed by pa_decode over the grown sequences.
+ *   "PagedAttention: KV cache as virtual memory", "Deep dive" (each decode
+ *   step appends one token, a new block when the last one is full) and the
+ *   pa_decode passages.
+ * Sequence s has ctx_lens[s] cached tokens; its new token's K/V rows
+ * (new_key / new_value T[num_seqs][num_kv_heads][head_dim]) are written to
+ * logical position ctx_lens[s] (slot block_tables[s][ctx / block_size] *
+ * block_size + ctx % block_size, bit copies), then out = attention of
+ * query[s] over the ctx_lens[s] + 1 tokens.  The writes are made by the CTAs
+ * that read that block, before they read it, so no second launch is needed.
+ * Output and cache contents are bit-identical to pa_append + pa_decode with
+ * seq_lens = ctx_lens + 1, max_seq_len = max_ctx_len + 1 and the same
+ * partition_tokens and workspace (pa_decode_workspace_size with
+ * max_ctx_len + 1).  slot_mapping (int64[num_seqs], may be NULL) receives
+ * the slot written, -1 when none (a block id outside the pool sets
+ * PA_DEVERR_BLOCK_RANGE; a context that does not fit the table sets
+ * PA_DEVERR_SEQ_RANGE and nothing is written).  fp16 / bf16 caches.
+ */
+pa_status pa_append_decode(void *out, const void *query, const void *new_key,
+                           const void *new_value, void *key_cache, void *value_cache,
+                           const int32_t *block_tables, const int32_t *ctx_lens,
+                           int64_t *slot_mapping, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_blocks_per_seq, int max_ctx_len, int partition_tokens,
+                           float scale, pa_dtype dtype, void *workspace, size_t workspace_bytes,
+                           pa_stream_t stream);
+
+/*
  * pa_decode_fp8 — pa_decode over FP8 (E4M3) caches (see pa_reshape_and_cache_fp8
  * for the encoding).  Attention is computed over the values code * k_scale and
  * code * v_scale; the query and output are fp16 or bf16 (`dtype`).  The

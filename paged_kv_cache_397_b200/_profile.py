@@ -29,15 +29,17 @@ import synth  # noqa: E402
 
 
 def decode_case(seqs: int, reps: int = 3):
+    """The bench's decode step (pa_append_decode) on a slice of its batch."""
     w = synth.llama3_8b_gqa_decode(num_seqs=seqs)
     d = torch.device("cuda:0")
     kc, vc, bt = w.key_cache.to(d), w.value_cache.to(d), w.block_tables.to(d)
-    lens = (w.context_lens + 1).to(d)
-    q = w.query.to(d)
+    ctx = w.context_lens.to(d)
+    lens = ctx + 1
+    q, nk, nv = w.query.to(d), w.new_key.to(d), w.new_value.to(d)
     out = torch.empty_like(q)
-    max_len = int(lens.max())
-    for _ in range(reps):
-        pa.pa_decode(out, q, kc, vc, bt, lens, max_len, w.scale)
+    max_ctx = int(w.context_lens.max())
+    for _ in range(reps):  # the same token rewritten into the same slot each time
+        pa.pa_append_decode(out, q, nk, nv, kc, vc, bt, ctx, max_ctx, w.scale)
     torch.cuda.synchronize()
     kv = 2 * w.num_kv_heads * w.head_dim * 2 * int(lens.sum())
     print(f"decode case: {w.name}, K/V bytes per launch {kv}")

@@ -62,6 +62,14 @@ struct DecodeParams {
   float scale_log2;          // softmax scale * log2(e) (FP8: also * k_scale)
   float v_scale;             // FP8: multiplies the output; 1 otherwise
   int len_add;               // tokens attended = seq_lens[s] + len_add (mixed batch: 1)
+  // Fused append (pa_append_decode; null otherwise): the new token of
+  // sequence s, at logical position seq_lens[s], is written into the cache
+  // by the CTAs of its last partition before they read that block.
+  const void* new_key;       // T[S][Hkv][D]
+  const void* new_value;     // T[S][Hkv][D]
+  void* key_cache;           // T[num_blocks][Hkv][BS][D]
+  void* value_cache;
+  int64_t* slot_out;         // [S] slot written (-1: none), or null
 };
 
 // ------------------------------------------------------------------ tiles
@@ -81,6 +89,7 @@ struct HalfTiles {
   static constexpr int BOXES = D / 64;              // TMA boxes per tile
   static constexpr int BOX_BYTES = BS * 128;
   static constexpr int HP = 1;                       // KV heads per ring stage
+  static constexpr bool kHalfCache = true;           // cache elements are T
   static constexpr int TILE_ROWS = BS;               // one cache block per ring stage
   static constexpr int TILE_BYTES = BS * D * 2;
   static constexpr int NS = BS == 16 ? 8 : 4;        // ring depth
@@ -206,6 +215,7 @@ struct E4m3Tiles {
   // 32-token blocks, against 4.6 TB/s for one 16-token block per stage at
   // four CTAs per SM and 3.5 TB/s for 32-token blocks with 4 stages.
   static constexpr int HP = HP_;
+  static constexpr bool kHalfCache = false;  // cache elements are E4M3 codes
   static constexpr int BOX_BYTES = HP * BS * 128;
   static constexpr int TILE_ROWS = 32;
   static constexpr int TILE_BYTES = TILE_ROWS * 128;
@@ -629,6 +639,36 @@ __device__ __forceinline__ void reset_state(float (&o)[Tiles::D / 16][NT][4],
   }
 }
 
+// Fused append, by the producer warp of the item that holds logical position
+// `pos` (the sequence's new token): write the token's K and V rows of KV
+// head kvh into its slot (block_tables[s][pos / BS], offset pos % BS), bit
+// copies, 16 bytes per lane, then order those writes before this CTA's TMA
+// reads of the block.  An out-of-pool block id is flagged and not written.
+template <class Tiles, int BS>
+__device__ __forceinline__ void append_new_token(const DecodeParams& p, int s, int kvh, int pos,
+                                                 int lane) {
+  constexpr int CH = Tiles::D * 2 / 16;  // 16-byte chunks per K or V row
+  const int32_t blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + pos / BS);
+  const bool ok = blk >= 0 && blk < p.num_blocks;
+  if (ok) {
+    const size_t row = ((size_t)blk * p.num_kv_heads + kvh) * BS + pos % BS;
+    const size_t src = (size_t)s * p.num_kv_heads + kvh;
+    for (int i = lane; i < 2 * CH; i += 32) {
+      const bool is_v = i >= CH;
+      const int c = is_v ? i - CH : i;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(is_v ? p.new_value : p.new_key) +
+                            src * CH + c);
+      reinterpret_cast<uint4*>(is_v ? p.value_cache : p.key_cache)[row * CH + c] = v;
+    }
+  } else if (lane == 0) {
+    record_error(PA_DEVERR_BLOCK_RANGE);
+  }
+  if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
+    p.slot_out[s] = ok ? (int64_t)blk * BS + pos % BS : -1;
+  fence_proxy_async_global();
+  __syncwarp();
+}
+
 // One work item (split-KV partition `part` of KV head `kvh` of sequence `s`)
 // run by THREADS consecutive threads (`tid` 0 .. THREADS-1) that own the
 // 1024-byte aligned shared memory at `smem` (SMEM_BYTES - 1024 bytes).  They
@@ -667,6 +707,16 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
     if (lane == 0) {
       tma_prefetch_desc(tm_k);
       tma_prefetch_desc(tm_v);
+    }
+    if constexpr (Tiles::kHalfCache) {
+      // fused append: the new token is the last position; skipped when the
+      // length was clamped (flagged by decode_len)
+      if (p.new_key != nullptr && part == nparts - 1) {
+        if (L >= 1 && p.seq_lens[s] + p.len_add == L)
+          append_new_token<Tiles, BS>(p, s, kvh, L - 1, lane);
+        else if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
+          p.slot_out[s] = -1;
+      }
     }
     produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s, kvh, blk0, nblk, 0,
                                 lane, l2_policy_evict_first(), true);

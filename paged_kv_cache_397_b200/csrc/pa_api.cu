@@ -488,13 +488,21 @@ namespace {
 
 // Validation, partition planning and launch shared by pa_decode (fp16 / bf16
 // caches) and pa_decode_fp8 (E4M3 caches, kv_fp8 = true).
+// The fused append of pa_append_decode (null for plain decode).
+struct AppendArgs {
+  const void* new_key;
+  const void* new_value;
+  int64_t* slot_out;
+};
+
 pa_status decode_impl(void* out, const void* query, const void* key_cache,
                       const void* value_cache, const int32_t* block_tables,
                       const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
                       int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
                       int max_seq_len, int partition_tokens, float scale, float k_scale,
                       float v_scale, bool kv_fp8, pa_dtype dtype, void* workspace,
-                      size_t workspace_bytes, pa_stream_t stream) {
+                      size_t workspace_bytes, pa_stream_t stream,
+                      const AppendArgs* app = nullptr) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
       max_blocks_per_seq <= 0 || max_seq_len < 0 || partition_tokens < 0 ||
       !valid_dtype(dtype) || !std::isfinite(scale))
@@ -507,6 +515,9 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
   if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens)
     return PA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if (app && (kv_fp8 || !app->new_key || !app->new_value || !aligned16(app->new_key) ||
+              !aligned16(app->new_value)))
     return PA_ERR_INVALID_ARG;
   if ((long long)max_seq_len > (long long)max_blocks_per_seq * block_size)
     return PA_ERR_INVALID_ARG;
@@ -558,7 +569,12 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
   p.max_parts = num_parts;
   p.scale_log2 = scale * (kv_fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   p.v_scale = kv_fp8 ? v_scale : 1.f;
-  p.len_add = 0;
+  p.len_add = app ? 1 : 0;  // fused append: seq_lens holds the context lengths
+  p.new_key = app ? app->new_key : nullptr;
+  p.new_value = app ? app->new_value : nullptr;
+  p.key_cache = app ? const_cast<void*>(key_cache) : nullptr;
+  p.value_cache = app ? const_cast<void*>(value_cache) : nullptr;
+  p.slot_out = app ? app->slot_out : nullptr;
   auto st = (cudaStream_t)stream;
   if (kv_fp8) {
     if (dtype == PA_BF16) return dispatch_decode_fp8<__nv_bfloat16>(block_size, mk, mv, p, num_parts, st);
@@ -583,6 +599,22 @@ pa_status pa_decode(void* out, const void* query, const void* key_cache, const v
                      num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                      max_blocks_per_seq, max_seq_len, partition_tokens, scale, 1.f, 1.f, false,
                      dtype, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_append_decode(void* out, const void* query, const void* new_key,
+                           const void* new_value, void* key_cache, void* value_cache,
+                           const int32_t* block_tables, const int32_t* ctx_lens,
+                           int64_t* slot_mapping, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_blocks_per_seq, int max_ctx_len, int partition_tokens,
+                           float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                           pa_stream_t stream) {
+  if (max_ctx_len < 0) return PA_ERR_INVALID_ARG;
+  const AppendArgs app{new_key, new_value, slot_mapping};
+  return decode_impl(out, query, key_cache, value_cache, block_tables, ctx_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                     max_blocks_per_seq, max_ctx_len + 1, partition_tokens, scale, 1.f, 1.f,
+                     false, dtype, workspace, workspace_bytes, stream, &app);
 }
 
 pa_status pa_decode_fp8(void* out, const void* query, const uint8_t* key_cache,
@@ -819,6 +851,9 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
   dp.block_tables = block_tables;
   dp.seq_lens = ctx_lens;
   dp.len_add = 1;
+  dp.new_key = dp.new_value = nullptr;
+  dp.key_cache = dp.value_cache = nullptr;
+  dp.slot_out = nullptr;
   uint8_t* ws_base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
   float* ws = reinterpret_cast<float*>(ws_base + 256);
