@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <mutex>
@@ -86,6 +87,30 @@ int sm_count() {
   return cached[dev];
 }
 
+// One-time per (kernel, device) launch configuration: the dynamic shared
+// memory limit is a per-device function attribute, so a process that drives
+// several GPUs must set it on each.  `min_regs` > 0 also refuses a build whose
+// kernel has fewer registers per thread than its setmaxnreg split needs (the
+// register increase could never be granted).
+template <typename K>
+pa_status configure_kernel(K kern, int smem_bytes, int min_regs) {
+  static std::atomic<unsigned long long> done{0};  // bit d: device d configured
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  const unsigned long long bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return PA_OK;
+  if (min_regs > 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return PA_ERR_CUDA;
+    if (attr.numRegs < min_regs) return PA_ERR_UNSUPPORTED;
+  }
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_release);
+  return PA_OK;
+}
+
 std::mutex g_static_ws_mutex;
 void* g_static_ws_addr[kMaxDevices] = {};
 
@@ -128,13 +153,7 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
   using Shape = pa::DecodeShape<Tiles, BS, NT>;
   using T = typename Tiles::Elem;
   auto kern = pa::decode_kernel<Tiles, BS, NT>;
-  static bool configured = false;  // per instantiation; attribute is per device-function
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Shape::SMEM_BYTES) != cudaSuccess)
-      return PA_ERR_CUDA;
-    configured = true;
-  }
+  if (pa_status st = configure_kernel(kern, Shape::SMEM_BYTES, 0); st != PA_OK) return st;
   dim3 grid(num_parts, p.num_kv_heads / Tiles::HP, p.num_seqs);  // y: packs of HP kv heads
   kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
@@ -224,19 +243,9 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
                       pa::PrefillParams p, cudaStream_t stream) {
   using Sh = pa::PrefillShape<T, BS>;
   auto kern = pa::prefill_kernel<T, BS>;
-  static bool configured = false;
-  if (!configured) {
-    // The kernel's setmaxnreg split assumes at least MIN_LAUNCH_REGS registers
-    // per thread at launch; with fewer, its register increase could never be
-    // granted, so such a build is refused rather than launched.
-    cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return PA_ERR_CUDA;
-    if (attr.numRegs < Sh::MIN_LAUNCH_REGS) return PA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Sh::SMEM_BYTES) != cudaSuccess)
-      return PA_ERR_CUDA;
-    configured = true;
-  }
+  // the kernel's setmaxnreg split assumes at least MIN_LAUNCH_REGS registers per thread
+  if (pa_status st = configure_kernel(kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS); st != PA_OK)
+    return st;
   const long long units = (long long)p.tiles_per_seq * p.num_q_heads * p.num_seqs;
   const long long grid = p.n_full + (units - p.n_full) * p.split;
   if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
@@ -273,18 +282,10 @@ pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
                     const pa::MixedPlan& plan, cudaStream_t stream) {
   using Sh = pa::MixedShape<T, BS, NT>;
   auto kern = pa::mixed_kernel<T, BS, NT>;
-  static bool configured = false;
-  if (!configured) {
-    // same register-split requirement as prefill_kernel (the prefill tiles
-    // of this kernel run the same setmaxnreg split)
-    cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return PA_ERR_CUDA;
-    if (attr.numRegs < Sh::MIN_LAUNCH_REGS) return PA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Sh::SMEM_BYTES) != cudaSuccess)
-      return PA_ERR_CUDA;
-    configured = true;
-  }
+  // same register-split requirement as prefill_kernel (its prefill tiles
+  // run the same setmaxnreg split)
+  if (pa_status st = configure_kernel(kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS); st != PA_OK)
+    return st;
   // persistent decode workers: at most one CTA (two workers) per SM
   long long decode_ctas = ((long long)plan.decode_items + Sh::WORKERS - 1) / Sh::WORKERS;
   if (decode_ctas > sm_count()) decode_ctas = sm_count();
