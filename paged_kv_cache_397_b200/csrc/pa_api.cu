@@ -89,12 +89,14 @@ int sm_count() {
 
 // One-time per (kernel, device) launch configuration: the dynamic shared
 // memory limit is a per-device function attribute, so a process that drives
-// several GPUs must set it on each.  `min_regs` > 0 also refuses a build whose
-// kernel has fewer registers per thread than its setmaxnreg split needs (the
-// register increase could never be granted).
+// several GPUs must set it on each.  `done` is the caller's per-kernel flag
+// word (bit d: device d configured): kernel instantiations share a function
+// type, so the flags cannot live in this template.  `min_regs` > 0 also
+// refuses a build whose kernel has fewer registers per thread than its
+// setmaxnreg split needs (the register increase could never be granted).
 template <typename K>
-pa_status configure_kernel(K kern, int smem_bytes, int min_regs) {
-  static std::atomic<unsigned long long> done{0};  // bit d: device d configured
+pa_status configure_kernel(std::atomic<unsigned long long>& done, K kern, int smem_bytes,
+                           int min_regs) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
   const unsigned long long bit = 1ull << dev;
@@ -153,7 +155,9 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
   using Shape = pa::DecodeShape<Tiles, BS, NT>;
   using T = typename Tiles::Elem;
   auto kern = pa::decode_kernel<Tiles, BS, NT>;
-  if (pa_status st = configure_kernel(kern, Shape::SMEM_BYTES, 0); st != PA_OK) return st;
+  static std::atomic<unsigned long long> configured{0};  // per instantiation
+  if (pa_status st = configure_kernel(configured, kern, Shape::SMEM_BYTES, 0); st != PA_OK)
+    return st;
   dim3 grid(num_parts, p.num_kv_heads / Tiles::HP, p.num_seqs);  // y: packs of HP kv heads
   kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
@@ -244,7 +248,9 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   using Sh = pa::PrefillShape<T, BS>;
   auto kern = pa::prefill_kernel<T, BS>;
   // the kernel's setmaxnreg split assumes at least MIN_LAUNCH_REGS registers per thread
-  if (pa_status st = configure_kernel(kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS); st != PA_OK)
+  static std::atomic<unsigned long long> configured{0};  // per instantiation
+  if (pa_status st = configure_kernel(configured, kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS);
+      st != PA_OK)
     return st;
   const long long units = (long long)p.tiles_per_seq * p.num_q_heads * p.num_seqs;
   const long long grid = p.n_full + (units - p.n_full) * p.split;
@@ -284,7 +290,9 @@ pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   auto kern = pa::mixed_kernel<T, BS, NT>;
   // same register-split requirement as prefill_kernel (its prefill tiles
   // run the same setmaxnreg split)
-  if (pa_status st = configure_kernel(kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS); st != PA_OK)
+  static std::atomic<unsigned long long> configured{0};  // per instantiation
+  if (pa_status st = configure_kernel(configured, kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS);
+      st != PA_OK)
     return st;
   // persistent decode workers: at most one CTA (two workers) per SM
   long long decode_ctas = ((long long)plan.decode_items + Sh::WORKERS - 1) / Sh::WORKERS;
