@@ -202,3 +202,71 @@ def test_random_churn_keeps_the_pool_consistent():
             for b in range(200):
                 assert bm.ref_count(b) == refs[b]
             assert bm.num_free_blocks == int((refs == 0).sum())
+
+
+@pytest.mark.parametrize("seed,B", [(1, 16), (2, 32), (3, 16)])
+def test_simulated_pool_reads_back_every_sequence(seed, B):
+    # The kernels' view of the manager: every token is written through the
+    # slots it hands out, copy-on-write pairs are applied before the writes of
+    # the step that needs them, and reading a sequence through its block table
+    # must give back exactly its tokens -- prefix hits, revived free blocks,
+    # forks and copy-on-write included ("PagedAttention: KV cache as virtual
+    # memory", "Deep dive").
+    rng = np.random.default_rng(seed)
+    nb = 160
+    bm = pa.BlockManager(nb, B)
+    pool = np.full((nb, B), -1, dtype=np.int64)  # token id held by each slot
+    seqs = {}
+    next_id = 0
+    prefixes = [toks(int(rng.integers(B, 6 * B)), 10_000 * k) for k in range(4)]
+
+    def write(sid, start, tokens):
+        if len(tokens) == 0:
+            return
+        for slot, t in zip(bm.slots(sid, start, len(tokens)), tokens):
+            pool[slot // B, slot % B] = t
+
+    def apply_copies():
+        for src, dst in bm.take_copies():
+            pool[dst] = pool[src]
+
+    for step in range(1500):
+        op = rng.random()
+        try:
+            if op < 0.3 or not seqs:
+                pre = prefixes[rng.integers(0, len(prefixes))]
+                cut = int(rng.integers(0, len(pre) + 1))
+                tail = toks(int(rng.integers(0, 2 * B)), 1_000_000 + 100 * step)
+                prompt = np.concatenate([pre[:cut], tail])
+                if len(prompt) == 0:
+                    continue
+                cached = bm.add_sequence(next_id, prompt)
+                apply_copies()
+                write(next_id, cached, prompt[cached:])
+                seqs[next_id] = list(prompt)
+                next_id += 1
+            elif op < 0.7:
+                sid = list(seqs)[rng.integers(0, len(seqs))]
+                new = toks(int(rng.integers(1, B + 3)), 5_000_000 + 100 * step)
+                bm.append(sid, new)
+                apply_copies()
+                write(sid, len(seqs[sid]), new)
+                seqs[sid] += list(new)
+            elif op < 0.82:
+                sid = list(seqs)[rng.integers(0, len(seqs))]
+                bm.fork(sid, next_id)
+                seqs[next_id] = list(seqs[sid])
+                next_id += 1
+            else:
+                sid = list(seqs)[rng.integers(0, len(seqs))]
+                bm.free(sid)
+                del seqs[sid]
+        except pa.PAError as e:
+            assert e.status == pa.PA_ERR_OUT_OF_RANGE  # pool exhausted; state unchanged
+        for sid, want in seqs.items():
+            table = bm.block_table(sid)
+            got = [pool[table[p // B], p % B] for p in range(len(want))]
+            assert got == want, f"sequence {sid} reads back wrong tokens at step {step}"
+    for sid in list(seqs):
+        bm.free(sid)
+    assert bm.num_free_blocks == nb
