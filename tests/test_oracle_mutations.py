@@ -1,0 +1,163 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of an oracle function (on the CPU),
+swaps it in for the real one, and checks that the pin written for that part
+of the oracle now fails: a scale applied twice, an off-by-one block index, an
+interleaved GQA grouping, an exclusive causal mask, a split-KV combine
+without the log-sum-exp rescale, a slot built from the wrong quotient, K and
+V swapped in the scatter, ties rounded away from the even E4M3 code, a KV
+byte count without the K/V factor, and a floor where the pages take a
+ceiling.  The real functions pass the same pins (they run in the rest of the
+suite)."""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.arithmetic as oa
+import oracle.fp8 as of
+import oracle.paged_attention as opa
+import test_oracle_arithmetic as t_arith
+import test_oracle_attention as t_attn
+import test_oracle_fp8 as t_fp8
+import test_oracle_indexing as t_idx
+from conftest import read_golden
+
+
+def _swap(monkeypatch, module, name, fn):
+    monkeypatch.setattr(module, name, fn)
+    if hasattr(oracle, name):
+        monkeypatch.setattr(oracle, name, fn)
+
+
+def _fails(pin, *args):
+    with pytest.raises(AssertionError):
+        pin(*args)
+
+
+def test_scale_applied_twice_is_caught(monkeypatch):
+    def attention(q, K, V, scale, visible=None):
+        q, K, V = (np.asarray(a, dtype=np.float64) for a in (q, K, V))
+        out = np.zeros((q.shape[0], V.shape[1]))
+        for m in range(q.shape[0]):
+            n = K.shape[0] if visible is None else int(visible[m])
+            if n > 0:
+                z = scale * scale * (K[:n] @ q[m])  # planted mistake
+                w = np.exp(z - z.max())
+                out[m] = (w @ V[:n]) / w.sum()
+        return out
+    _swap(monkeypatch, opa, "attention", attention)
+    _fails(t_attn.test_decode_equals_dense_sdpa, 16, 8, 2, 100)
+
+
+def test_off_by_one_block_index_is_caught(monkeypatch):
+    def gather_logical(cache, table_row, length, kv_head, block_size):
+        p = np.arange(int(length))
+        phys = np.asarray(table_row)[(p + 1) // block_size]  # planted mistake
+        return np.asarray(cache[phys, kv_head, p % block_size, :], dtype=np.float64)
+    _swap(monkeypatch, opa, "gather_logical", gather_logical)
+    _fails(t_attn.test_decode_equals_dense_sdpa, 16, 4, 4, 17)
+
+
+def test_interleaved_gqa_grouping_is_caught(monkeypatch):
+    def paged_decode(query, key_cache, value_cache, block_tables, seq_lens, scale, num_kv_heads):
+        q = np.asarray(query, dtype=np.float64)
+        S, Hq, D = q.shape
+        B = key_cache.shape[2]
+        out = np.zeros((S, Hq, D))
+        for s in range(S):
+            for h in range(Hq):
+                g = h % num_kv_heads  # planted mistake (contiguous groups: h // G)
+                K = opa.gather_logical(key_cache, block_tables[s], seq_lens[s], g, B)
+                V = opa.gather_logical(value_cache, block_tables[s], seq_lens[s], g, B)
+                out[s, h] = opa.attention(q[s, h][None], K, V, scale)[0]
+        return out
+    _swap(monkeypatch, opa, "paged_decode", paged_decode)
+    _fails(t_attn.test_decode_gqa_grouping_is_contiguous)
+
+
+def test_exclusive_causal_mask_is_caught(monkeypatch):
+    real = opa.paged_prefill_chunk
+
+    def paged_prefill_chunk(query, key_cache, value_cache, block_tables, cu_q_lens, ctx_lens,
+                            scale, num_kv_heads, seqs=None, rows=None):
+        q = np.asarray(query, dtype=np.float64)
+        T, Hq, D = q.shape
+        B = key_cache.shape[2]
+        G = Hq // num_kv_heads
+        out = np.zeros((T, Hq, D))
+        for s in range(len(ctx_lens)):
+            q0, q1, c = int(cu_q_lens[s]), int(cu_q_lens[s + 1]), int(ctx_lens[s])
+            idx = np.arange(q1 - q0)
+            if idx.size == 0:
+                continue
+            L = c + idx.size
+            for g in range(num_kv_heads):
+                K = opa.gather_logical(key_cache, block_tables[s], L, g, B)
+                V = opa.gather_logical(value_cache, block_tables[s], L, g, B)
+                for h in range(g * G, (g + 1) * G):
+                    # planted mistake: row i does not see itself
+                    out[q0 + idx, h] = opa.attention(q[q0 + idx, h], K, V, scale,
+                                                     visible=c + idx)
+        return out
+    assert real is not paged_prefill_chunk
+    _swap(monkeypatch, opa, "paged_prefill_chunk", paged_prefill_chunk)
+    _fails(t_attn.test_prefill_chunk_equals_masked_sdpa, 16)
+
+
+def test_combine_without_rescale_is_caught(monkeypatch):
+    def combine_partials(states):
+        num = sum(acc for m, l, acc in states if not np.isneginf(m))  # planted mistake
+        den = sum(l for m, l, acc in states if not np.isneginf(m))
+        return num / den
+    _swap(monkeypatch, opa, "combine_partials", combine_partials)
+    _fails(t_attn.test_split_kv_combine_equals_unsplit, [16, 17])
+
+
+def test_slot_offset_from_the_wrong_quotient_is_caught(monkeypatch):
+    def logical_positions_to_slots(block_tables, seq_ids, positions, block_size):
+        bt = np.asarray(block_tables, dtype=np.int64)
+        s = np.asarray(seq_ids, dtype=np.int64).reshape(-1)
+        p = np.asarray(positions, dtype=np.int64).reshape(-1)
+        return bt[s, p // block_size] * block_size + p // block_size  # planted mistake
+    _swap(monkeypatch, opa, "logical_positions_to_slots", logical_positions_to_slots)
+    _fails(t_idx.test_slots_of_the_worked_example, read_golden)
+
+
+def test_key_value_swap_in_the_scatter_is_caught(monkeypatch):
+    def reshape_and_cache(key_cache, value_cache, key, value, slot_mapping, block_size):
+        for t, slot in enumerate(np.asarray(slot_mapping).reshape(-1)):
+            if slot >= 0:
+                key_cache[slot // block_size, :, slot % block_size, :] = value[t]  # planted
+                value_cache[slot // block_size, :, slot % block_size, :] = key[t]
+    _swap(monkeypatch, opa, "reshape_and_cache", reshape_and_cache)
+    _fails(t_idx.test_reshape_and_cache_bits_and_skip)
+
+
+def test_ties_away_from_even_are_caught(monkeypatch):
+    values = of._POS_VALUES
+
+    def e4m3_encode(x):
+        x = np.asarray(x, dtype=np.float64)
+        mag = np.minimum(np.abs(np.nan_to_num(x)), values[0x7E])
+        hi = np.minimum(np.searchsorted(values, mag, side="left"), 0x7E)
+        lo = np.maximum(np.where(values[hi] > mag, hi - 1, hi), 0)
+        pick_hi = (values[hi] - mag) <= (mag - values[lo])  # planted mistake: ties go up
+        code = np.where(pick_hi, hi, lo).astype(np.uint8)
+        code = np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)
+        return np.where(np.isnan(x), np.uint8(0x7F), code).astype(np.uint8)
+    _swap(monkeypatch, of, "e4m3_encode", e4m3_encode)
+    _fails(t_fp8.test_ties_go_to_the_even_code)
+
+
+def test_kv_bytes_without_the_kv_factor_is_caught(monkeypatch):
+    def kv_bytes_per_token(num_layers, num_kv_heads, head_dim, dtype_bytes):
+        return num_layers * num_kv_heads * head_dim * dtype_bytes  # planted mistake
+    _swap(monkeypatch, oa, "kv_bytes_per_token", kv_bytes_per_token)
+    _fails(t_arith.test_kv_bytes_per_token_llama2_13b, read_golden)
+
+
+def test_floor_instead_of_ceiling_is_caught(monkeypatch):
+    def blocks_needed(num_tokens, block_size):
+        return num_tokens // block_size  # planted mistake
+    _swap(monkeypatch, oa, "blocks_needed", blocks_needed)
+    _fails(t_arith.test_block_table_example_counts, read_golden)
