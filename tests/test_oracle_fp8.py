@@ -74,6 +74,33 @@ def test_quantize_divides_in_fp32():
     np.testing.assert_array_equal(fp8.quantize(x.numpy(), scale), want.numpy())
 
 
+def _tie_inputs(scale):
+    # x whose fp32 quotient x / scale is exactly the midpoint of two adjacent
+    # normal E4M3 values while the exact (fp64) quotient is not: writing
+    # rounds the fp32 quotient, so these go to the even code
+    vals = fp8.E4M3_TABLE[:0x7F].astype(np.float64)
+    out = []
+    for i in range(8, 0x7E):
+        m = (vals[i] + vals[i + 1]) / 2
+        x = np.float32(m * float(scale))
+        for _ in range(64):
+            x = np.nextafter(x, np.float32(-np.inf))
+        for _ in range(129):
+            if float(np.float32(x) / scale) == m and float(x) / float(scale) != m:
+                out.append(x)
+            x = np.nextafter(x, np.float32(np.inf))
+    return np.array(out, dtype=np.float32)
+
+
+def test_quantize_divides_in_fp32_at_ties():
+    scale = np.float32(0.0371)
+    x = _tie_inputs(scale)
+    assert len(x) > 50
+    want = (torch.from_numpy(x) / torch.tensor(float(scale), dtype=torch.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    np.testing.assert_array_equal(fp8.quantize(x, float(scale)), want.numpy())
+
+
 def test_fp8_decode_is_decode_of_the_dequantized_cache():
     rng = np.random.default_rng(3)
     nb, hkv, B, D = 6, 2, 16, 8

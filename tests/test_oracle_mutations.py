@@ -6,9 +6,10 @@ of the oracle now fails: a scale applied twice, an off-by-one block index, an
 interleaved GQA grouping, an exclusive causal mask, a split-KV combine
 without the log-sum-exp rescale, a slot built from the wrong quotient, K and
 V swapped in the scatter, ties rounded away from the even E4M3 code, a KV
-byte count without the K/V factor, and a floor where the pages take a
-ceiling.  The real functions pass the same pins (they run in the rest of the
-suite)."""
+byte count without the K/V factor, a floor where the pages take a ceiling,
+a block copy in the wrong direction, a swap of one pool only, admission that
+never skips, FP8 quantisation dividing in fp64, and an off-by-one tail waste.
+The real functions pass the same pins (they run in the rest of the suite)."""
 import numpy as np
 import pytest
 
@@ -161,3 +162,49 @@ def test_floor_instead_of_ceiling_is_caught(monkeypatch):
         return num_tokens // block_size  # planted mistake
     _swap(monkeypatch, oa, "blocks_needed", blocks_needed)
     _fails(t_arith.test_block_table_example_counts, read_golden)
+
+
+def test_copy_in_the_wrong_direction_is_caught(monkeypatch):
+    def copy_blocks(key_cache, value_cache, block_pairs):
+        for src, dst in np.asarray(block_pairs, dtype=np.int64).reshape(-1, 2):
+            key_cache[src] = key_cache[dst]  # planted mistake: dst -> src
+            value_cache[src] = value_cache[dst]
+    _swap(monkeypatch, opa, "copy_blocks", copy_blocks)
+    _fails(t_idx.test_copy_blocks_bits)
+
+
+def test_swap_of_one_pool_only_is_caught(monkeypatch):
+    def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, block_pairs):
+        for src, dst in np.asarray(block_pairs, dtype=np.int64).reshape(-1, 2):
+            dst_key_cache[dst] = src_key_cache[src]  # planted mistake: V not swapped
+    _swap(monkeypatch, opa, "swap_blocks", swap_blocks)
+    _fails(t_idx.test_swap_blocks_copies_between_pools_only_the_listed_blocks)
+
+
+def test_admission_that_never_skips_is_caught(monkeypatch):
+    def paged_fit(lengths, pool_blocks, block_size, stop_at_first_miss):
+        used = admitted = 0
+        for L in lengths:
+            need = oa.blocks_needed(int(L), block_size)
+            if used + need > pool_blocks:
+                break  # planted mistake: both readings stop at the first miss
+            used += need
+            admitted += 1
+        return admitted
+    _swap(monkeypatch, oa, "paged_fit", paged_fit)
+    _fails(t_arith.test_fragmentation_fit, read_golden)
+
+
+def test_quantize_in_double_precision_is_caught(monkeypatch):
+    def quantize(x, scale):
+        q = np.asarray(x, dtype=np.float64) / float(scale)  # planted mistake: fp64 division
+        return of.e4m3_encode(q)
+    _swap(monkeypatch, of, "quantize", quantize)
+    _fails(t_fp8.test_quantize_divides_in_fp32_at_ties)
+
+
+def test_tail_waste_off_by_one_is_caught(monkeypatch):
+    def tail_waste_tokens(num_tokens, block_size):
+        return oa.blocks_needed(num_tokens, block_size) * block_size - num_tokens + 1  # planted
+    _swap(monkeypatch, oa, "tail_waste_tokens", tail_waste_tokens)
+    _fails(t_arith.test_tail_waste_bound_exhaustive, read_golden)
