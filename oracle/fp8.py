@@ -5,8 +5,7 @@ this module; the CUDA library never does.
 
 The pages name an FP8 KV cache as the way to halve bytes per block and raise
 concurrency ("PagedAttention: KV cache as virtual memory", "Deep dive" and
-"Interviewer follow-ups") but fix no format or scaling.  Readings (listed in
-DESIGN.md):
+"Interviewer follow-ups") but fix no format or scaling.  Readings taken:
   * the OCP 8-bit E4M3 encoding without infinities: 1 sign bit, 4 exponent
     bits (bias 7), 3 mantissa bits; exponent 0 is subnormal (m/8 * 2^-6);
     S.1111.111 is NaN; the largest finite value is 448;

@@ -20,7 +20,7 @@ Mechanism"), and the result is identical to dense attention ([Block Mgr]
 "Direct answer" and "Interviewer follow-ups").  So this oracle is dense softmax
 attention on the logically contiguous K/V each block table defines.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent (the library takes the same ones):
   * cache layout ``[num_blocks][num_kv_heads][block_size][head_dim]``, K and V
     in separate pools; slot of logical position p = table[p // B] * B + p % B;
     slot -1 means "skip";
