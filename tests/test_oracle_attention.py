@@ -285,6 +285,36 @@ def test_split_kv_combine_equals_unsplit(cuts):
     np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
 
 
+@pytest.mark.parametrize("parts", [2, 3, 4])
+def test_causal_chunk_rows_from_key_range_parts(parts):
+    # A chunk row split along the key range into equal runs of 128-key tiles
+    # (the last wave's split of the prefill kernel): each part keeps only the
+    # keys the row may see, a part with none contributes (-inf, 0, 0), and the
+    # parts' combine equals the row's causal attention.
+    w = synth.chunked_prefill(seed=21 + parts, block_size=16, hq=2, hkv=1, d=16,
+                              ctx_lens=[300], q_lens=[90], dtype=torch.float16)
+    kc = w.key_cache.double().numpy()
+    vc = w.value_cache.double().numpy()
+    q = w.query.double().numpy()
+    bt = w.block_tables.numpy()
+    c, n = 300, 90
+    whole = oracle.paged_prefill_chunk(q, kc, vc, bt, w.cu_q_lens.numpy(), [c], w.scale, 1)
+    L = c + n
+    K = oracle.gather_logical(kc, bt[0], L, 0, 16)
+    V = oracle.gather_logical(vc, bt[0], L, 0, 16)
+    ntiles = -(-L // 128)
+    for i in (0, 1, 45, 89):
+        for h in range(2):
+            states = []
+            for part in range(parts):
+                a = part * ntiles // parts * 128
+                b = min((part + 1) * ntiles // parts * 128, c + i + 1)  # causal limit
+                states.append(oracle.partial_attention(q[i, h], K[a:max(a, b)], V[a:max(a, b)],
+                                                       w.scale))
+            np.testing.assert_allclose(oracle.combine_partials(states), whole[i, h], atol=1e-12,
+                                       rtol=0)
+
+
 def test_split_kv_partial_state_definition():
     rng = np.random.default_rng(9)
     K = rng.standard_normal((5, 4))
