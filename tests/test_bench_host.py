@@ -59,3 +59,19 @@ def test_traffic_is_reported_only_for_the_profiled_kernel_source(tmp_path, monke
     prof.write_text("dram_bytes_per_algorithmic_byte: 1.25000\n"
                     "kernel_source_sha256_16: 0000000000000000\n")
     assert bench.profiled_traffic(1000.0) is None
+
+
+def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
+    import argparse
+
+    import bench
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    assert bench.run_reference(argparse.Namespace(steps=2, warmup=3)) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
