@@ -101,3 +101,18 @@ def test_paged_fit_brute_force_small():
                     break
                 used, first = used + need, first + 1
             assert ar.paged_fit(lens, pool, 16, True) == first
+
+
+def test_contiguous_fit_brute_force():
+    # each admitted sequence takes whole blocks for max_len tokens up front;
+    # admit until the next reservation no longer fits in what is left
+    for B in (1, 4, 16):
+        for max_len in range(1, 40):
+            need = -(-max_len // B)
+            for pool in range(0, 30):
+                free = pool
+                n = 0
+                while need <= free:
+                    free -= need
+                    n += 1
+                assert ar.contiguous_fit(pool, max_len, B) == n

@@ -8,7 +8,12 @@ without the log-sum-exp rescale, a slot built from the wrong quotient, K and
 V swapped in the scatter, ties rounded away from the even E4M3 code, a KV
 byte count without the K/V factor, a floor where the pages take a ceiling,
 a block copy in the wrong direction, a swap of one pool only, admission that
-never skips, FP8 quantisation dividing in fp64, and an off-by-one tail waste.
+never skips, FP8 quantisation dividing in fp64, an off-by-one tail waste, a
+contiguous reservation counted in tokens rather than whole blocks, the waste
+share inverted, an E4M3 exponent bias of 8, a subnormal step of 2^-10, V
+dequantised with the K scale, a partial state already normalised, a chunk
+whose rows ignore the cached context, overflow to NaN instead of saturation,
+and a skipped slot (-1) written to the last block.
 The real functions pass the same pins (they run in the rest of the suite)."""
 import numpy as np
 import pytest
@@ -76,9 +81,8 @@ def test_interleaved_gqa_grouping_is_caught(monkeypatch):
     _fails(t_attn.test_decode_gqa_grouping_is_contiguous)
 
 
-def test_exclusive_causal_mask_is_caught(monkeypatch):
-    real = opa.paged_prefill_chunk
-
+def _chunk_with_visible(visible_of):
+    """paged_prefill_chunk with the keys row i may see given by visible_of(c, i)."""
     def paged_prefill_chunk(query, key_cache, value_cache, block_tables, cu_q_lens, ctx_lens,
                             scale, num_kv_heads, seqs=None, rows=None):
         q = np.asarray(query, dtype=np.float64)
@@ -96,12 +100,21 @@ def test_exclusive_causal_mask_is_caught(monkeypatch):
                 K = opa.gather_logical(key_cache, block_tables[s], L, g, B)
                 V = opa.gather_logical(value_cache, block_tables[s], L, g, B)
                 for h in range(g * G, (g + 1) * G):
-                    # planted mistake: row i does not see itself
                     out[q0 + idx, h] = opa.attention(q[q0 + idx, h], K, V, scale,
-                                                     visible=c + idx)
+                                                     visible=visible_of(c, idx))
         return out
-    assert real is not paged_prefill_chunk
-    _swap(monkeypatch, opa, "paged_prefill_chunk", paged_prefill_chunk)
+    return paged_prefill_chunk
+
+
+def test_exclusive_causal_mask_is_caught(monkeypatch):
+    # planted mistake: row i does not see itself
+    _swap(monkeypatch, opa, "paged_prefill_chunk", _chunk_with_visible(lambda c, i: c + i))
+    _fails(t_attn.test_prefill_chunk_equals_masked_sdpa, 16)
+
+
+def test_chunk_that_ignores_the_context_is_caught(monkeypatch):
+    # planted mistake: row i is placed at position i, not after the c cached tokens
+    _swap(monkeypatch, opa, "paged_prefill_chunk", _chunk_with_visible(lambda c, i: i + 1))
     _fails(t_attn.test_prefill_chunk_equals_masked_sdpa, 16)
 
 
@@ -208,3 +221,79 @@ def test_tail_waste_off_by_one_is_caught(monkeypatch):
         return oa.blocks_needed(num_tokens, block_size) * block_size - num_tokens + 1  # planted
     _swap(monkeypatch, oa, "tail_waste_tokens", tail_waste_tokens)
     _fails(t_arith.test_tail_waste_bound_exhaustive, read_golden)
+
+
+def test_contiguous_fit_in_tokens_is_caught(monkeypatch):
+    def contiguous_fit(pool_blocks, max_len, block_size):
+        return pool_blocks * block_size // max_len  # planted mistake: reservation not whole blocks
+    _swap(monkeypatch, oa, "contiguous_fit", contiguous_fit)
+    _fails(t_arith.test_contiguous_fit_brute_force)
+
+
+def test_inverted_waste_share_is_caught(monkeypatch):
+    def reservation_waste_fraction(tokens_used, tokens_reserved):
+        return tokens_used / tokens_reserved  # planted mistake: the used share
+    _swap(monkeypatch, oa, "reservation_waste_fraction", reservation_waste_fraction)
+    _fails(t_arith.test_reservation_waste, read_golden)
+
+
+@pytest.mark.parametrize("bias,sub_exp", [(8, -6), (7, -7)])
+def test_wrong_e4m3_code_values_are_caught(monkeypatch, bias, sub_exp):
+    def e4m3_value(code):
+        code = int(code) & 0xFF
+        s = -1.0 if code & 0x80 else 1.0
+        e, m = (code >> 3) & 0xF, code & 0x7
+        if e == 0xF and m == 0x7:
+            return float("nan")
+        if e == 0:
+            return s * (m / 8.0) * 2.0 ** sub_exp  # planted mistake when sub_exp != -6
+        return s * (1.0 + m / 8.0) * 2.0 ** (e - bias)  # planted mistake when bias != 7
+    table = np.array([e4m3_value(c) for c in range(256)])
+    _swap(monkeypatch, of, "e4m3_value", e4m3_value)
+    monkeypatch.setattr(of, "E4M3_TABLE", table)
+    monkeypatch.setattr(of, "_POS_VALUES", table[:0x7F])
+    _fails(t_fp8.test_code_values_closed_forms)
+
+
+def test_values_dequantised_with_the_key_scale_are_caught(monkeypatch):
+    def paged_decode_fp8(query, key_codes, value_codes, block_tables, seq_lens, scale, k_scale,
+                         v_scale, num_kv_heads):
+        kc = of.E4M3_TABLE[np.asarray(key_codes, dtype=np.uint8)] * float(np.float32(k_scale))
+        vc = of.E4M3_TABLE[np.asarray(value_codes, dtype=np.uint8)] * float(np.float32(k_scale))
+        return opa.paged_decode(query, kc, vc, block_tables, seq_lens, scale, num_kv_heads)
+    _swap(monkeypatch, of, "paged_decode_fp8", paged_decode_fp8)
+    _fails(t_fp8.test_fp8_decode_is_decode_of_the_dequantized_cache)
+
+
+def test_normalised_partial_state_is_caught(monkeypatch):
+    def partial_attention(q, K, V, scale):
+        q = np.asarray(q, dtype=np.float64)
+        if K.shape[0] == 0:
+            return -np.inf, 0.0, np.zeros(V.shape[1])
+        z = scale * (np.asarray(K, dtype=np.float64) @ q)
+        w = np.exp(z - z.max())
+        return z.max(), w.sum(), (w @ np.asarray(V, dtype=np.float64)) / w.sum()  # planted
+    _swap(monkeypatch, opa, "partial_attention", partial_attention)
+    _fails(t_attn.test_split_kv_combine_equals_unsplit, [16, 17])
+
+
+def test_overflow_to_nan_is_caught(monkeypatch):
+    real = of.e4m3_encode
+
+    def e4m3_encode(x):
+        x = np.asarray(x, dtype=np.float64)
+        code = real(x)
+        # planted mistake: magnitudes above 448 become NaN instead of saturating
+        return np.where(np.abs(x) > 448.0, (code & 0x80) | 0x7F, code).astype(np.uint8)
+    _swap(monkeypatch, of, "e4m3_encode", e4m3_encode)
+    _fails(t_fp8.test_saturation_and_nan)
+
+
+def test_skipped_slot_written_is_caught(monkeypatch):
+    def reshape_and_cache(key_cache, value_cache, key, value, slot_mapping, block_size):
+        for t, slot in enumerate(np.asarray(slot_mapping).reshape(-1)):
+            slot = int(slot)  # planted mistake: -1 is not skipped (lands in the last block)
+            key_cache[slot // block_size, :, slot % block_size, :] = key[t]
+            value_cache[slot // block_size, :, slot % block_size, :] = value[t]
+    _swap(monkeypatch, opa, "reshape_and_cache", reshape_and_cache)
+    _fails(t_idx.test_reshape_and_cache_bits_and_skip)
