@@ -414,52 +414,72 @@ typedef struct pa_block_manager pa_block_manager;
 
 /* Pool of num_blocks blocks of block_size tokens; enable_prefix_caching != 0
  * turns on full-block prefix sharing.  Blocks are handed out 0, 1, 2, ...
- * while the pool is fresh. */
+ * while the pool is fresh.  PA_ERR_INVALID_ARG (nothing created) for a null
+ * `out`, a non-positive size, num_blocks * block_size above INT32_MAX (token
+ * counts and positions are int), or when the host tables cannot be
+ * allocated.  The handle is owned by the caller until pa_bm_destroy. */
 pa_status pa_bm_create(int num_blocks, int block_size, int enable_prefix_caching,
                        pa_block_manager **out);
 void pa_bm_destroy(pa_block_manager *bm);
 
-/* Admit a sequence with its prompt tokens: leading full blocks whose prefix
- * key is cached are shared (reference count + 1, revived from the free queue
- * if needed); the rest come from the front of the free queue.  Writes the
- * number of prompt tokens whose K/V are already cached.  PA_ERR_OUT_OF_RANGE
- * (state unchanged) when the pool cannot hold the prompt. */
+/* Admit a sequence with its prompt tokens (tokens[num_tokens], host memory,
+ * read during the call only): leading full blocks whose prefix key is cached
+ * are shared (reference count + 1, revived from the free queue if needed);
+ * the rest come from the front of the free queue.  Writes the number of
+ * prompt tokens whose K/V are already cached (num_cached_tokens may be NULL).
+ * PA_ERR_INVALID_ARG for an id already in use, a negative count or a null
+ * `tokens` with num_tokens > 0; PA_ERR_OUT_OF_RANGE when the pool cannot hold
+ * the prompt.  State is unchanged on every error. */
 pa_status pa_bm_add_sequence(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens,
                              int num_tokens, int *num_cached_tokens);
 
 /* Append generated tokens.  A new block is taken whenever the last one is
  * full.  If the last block is partially filled and shared (count > 1), it is
  * first replaced by a fresh block and the (src, dst) pair is queued for
- * pa_bm_take_copies (copy-on-write).  PA_ERR_OUT_OF_RANGE (state unchanged)
- * when the pool runs out. */
+ * pa_bm_take_copies (copy-on-write).  PA_ERR_INVALID_ARG for an unknown id, a
+ * negative count or a null `tokens` with num_tokens > 0; PA_ERR_OUT_OF_RANGE
+ * when the pool runs out.  State is unchanged on every error. */
 pa_status pa_bm_append(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens,
                        int num_tokens);
 
-/* The child shares every block of the parent (parallel sampling, beam search). */
+/* The child shares every block of the parent (parallel sampling, beam search).
+ * PA_ERR_INVALID_ARG (state unchanged) for an unknown parent or a child id
+ * already in use. */
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id);
 
 /* Finish a sequence: every block's count drops by one; blocks reaching zero
  * go to the back of the free queue, last logical block first.  Cached full
- * blocks keep their key until reused, so later prompts can still hit them. */
+ * blocks keep their key until reused, so later prompts can still hit them.
+ * PA_ERR_INVALID_ARG for an unknown id. */
 pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id);
 
-/* The sequence's physical blocks in logical order into out[capacity] (the
- * rest filled with -1); PA_ERR_WORKSPACE if capacity is too small. */
+/* The sequence's physical blocks in logical order into out[capacity] (host
+ * memory; the rest filled with -1).  *num_blocks (may be NULL) gets the
+ * table's length even when capacity is too small, which returns
+ * PA_ERR_WORKSPACE and writes nothing to `out`.  PA_ERR_INVALID_ARG for an
+ * unknown id, a negative capacity or a null `out` with capacity > 0. */
 pa_status pa_bm_block_table(const pa_block_manager *bm, int64_t seq_id, int32_t *out,
                             int capacity, int *num_blocks);
 
-/* Slots of logical positions start .. start + count - 1 (physical * B + offset). */
+/* Slots of logical positions start .. start + count - 1 (physical * B + offset)
+ * into out[count] (host memory).  Positions may run past the tokens held, up
+ * to the end of the sequence's last block; beyond it PA_ERR_OUT_OF_RANGE and
+ * nothing is written.  PA_ERR_INVALID_ARG for an unknown id, a negative start
+ * or count, or a null `out` with count > 0. */
 pa_status pa_bm_slots(const pa_block_manager *bm, int64_t seq_id, int start, int count,
                       int64_t *out);
 
-/* Move the queued copy-on-write pairs into pairs[capacity][2] and return how
- * many; returns minus the number pending (and takes none) if capacity is
- * too small. */
+/* Move the queued copy-on-write pairs into pairs[capacity][2] (host memory,
+ * (src, dst) in queue order) and return how many; returns minus the number
+ * pending (and takes none) if capacity is too small, and -1 for a null
+ * manager, a negative capacity or a null `pairs` with capacity > 0. */
 int pa_bm_take_copies(pa_block_manager *bm, int64_t *pairs, int capacity);
 
+/* Counters; each returns -1 for a null manager, an out-of-range block or an
+ * unknown sequence id. */
 int pa_bm_num_free_blocks(const pa_block_manager *bm);
 int pa_bm_ref_count(const pa_block_manager *bm, int block);
-int pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id); /* -1 if unknown */
+int pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id);
 
 /*
  * pa_get_device_error — synchronise `stream`, then read and clear the device

@@ -23,8 +23,9 @@
 //    appending into a partially filled block that is shared (count > 1, e.g.
 //    after fork) first copies it to a fresh block — copy-on-write — and
 //    queues the (src, dst) pair for pa_copy_blocks.
-// Keys are verified against the stored tokens on a hit, so a hash collision
-// can never alias two different prefixes.
+// A hit also compares the block's stored tokens, so two prefixes can share a
+// block only if that block's tokens are equal and the 64-bit keys of their
+// parents collide.
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -145,13 +146,20 @@ extern "C" {
 pa_status pa_bm_create(int num_blocks, int block_size, int enable_prefix_caching,
                        pa_block_manager** out) {
   if (!out || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+  // token counts and positions are int throughout the ABI
+  if ((int64_t)num_blocks * block_size > INT32_MAX) return PA_ERR_INVALID_ARG;
   auto* m = new (std::nothrow) pa_block_manager();
   if (!m) return PA_ERR_INVALID_ARG;
   m->num_blocks = num_blocks;
   m->block_size = block_size;
   m->prefix = enable_prefix_caching != 0;
-  m->blocks.resize(num_blocks);
-  if (m->prefix) m->cached_tokens.resize((size_t)num_blocks * block_size);
+  try {
+    m->blocks.resize(num_blocks);
+    if (m->prefix) m->cached_tokens.resize((size_t)num_blocks * block_size);
+  } catch (const std::bad_alloc&) {
+    delete m;
+    return PA_ERR_INVALID_ARG;
+  }
   for (int b = 0; b < num_blocks; ++b) m->push_back(b);  // ids in order: 0 is handed out first
   *out = m;
   return PA_OK;
@@ -177,7 +185,8 @@ pa_status pa_bm_add_sequence(pa_block_manager* m, int64_t seq_id, const int32_t*
   if (!m || num_tokens < 0 || (num_tokens > 0 && !tokens)) return PA_ERR_INVALID_ARG;
   if (m->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
   const int B = m->block_size;
-  const int need = (num_tokens + B - 1) / B;
+  const int64_t need = ((int64_t)num_tokens + B - 1) / B;
+  if (need > m->num_blocks) return PA_ERR_OUT_OF_RANGE;  // can never fit
   // leading full blocks already cached (prefix hits stop at the first miss)
   std::vector<int32_t> hits;
   std::vector<uint64_t> keys;
@@ -196,7 +205,7 @@ pa_status pa_bm_add_sequence(pa_block_manager* m, int64_t seq_id, const int32_t*
   // hits that sit in the free queue leave it, so count what must come from it
   int revived = 0;
   for (int32_t b : hits) revived += m->blocks[b].in_free ? 1 : 0;
-  const int fresh = need - (int)hits.size();
+  const int fresh = (int)need - (int)hits.size();
   if (fresh + revived > m->num_free) return PA_ERR_OUT_OF_RANGE;  // nothing changed
   Seq q;
   q.tokens.assign(tokens, tokens + num_tokens);
@@ -224,11 +233,11 @@ pa_status pa_bm_append(pa_block_manager* m, int64_t seq_id, const int32_t* token
   if (it == m->seqs.end()) return PA_ERR_INVALID_ARG;
   Seq& q = it->second;
   const int B = m->block_size;
-  const int L = (int)q.tokens.size();
+  const int64_t L = (int64_t)q.tokens.size();
   // blocks needed: a copy of a shared partial last block, plus new blocks
   const bool partial = L % B != 0;
   const bool cow = num_tokens > 0 && partial && m->blocks[q.table.back()].ref > 1;
-  const int new_blocks = (L + num_tokens + B - 1) / B - (L + B - 1) / B;
+  const int64_t new_blocks = (L + num_tokens + B - 1) / B - (L + B - 1) / B;
   if ((cow ? 1 : 0) + new_blocks > m->num_free) return PA_ERR_OUT_OF_RANGE;
   if (cow) {
     const int32_t src = q.table.back();
@@ -273,7 +282,7 @@ pa_status pa_bm_block_table(const pa_block_manager* m, int64_t seq_id, int32_t* 
   const std::vector<int32_t>& t = it->second.table;
   if (num_blocks) *num_blocks = (int)t.size();
   if ((int)t.size() > capacity) return PA_ERR_WORKSPACE;
-  std::memcpy(out, t.data(), sizeof(int32_t) * t.size());
+  if (!t.empty()) std::memcpy(out, t.data(), sizeof(int32_t) * t.size());
   for (int i = (int)t.size(); i < capacity; ++i) out[i] = -1;
   return PA_OK;
 }
@@ -284,7 +293,7 @@ pa_status pa_bm_slots(const pa_block_manager* m, int64_t seq_id, int start, int 
   auto it = m->seqs.find(seq_id);
   if (it == m->seqs.end()) return PA_ERR_INVALID_ARG;
   const Seq& q = it->second;
-  if (start + count > (int)q.table.size() * m->block_size) return PA_ERR_OUT_OF_RANGE;
+  if ((int64_t)start + count > (int64_t)q.table.size() * m->block_size) return PA_ERR_OUT_OF_RANGE;
   for (int i = 0; i < count; ++i) {
     const int p = start + i;
     out[i] = (int64_t)q.table[p / m->block_size] * m->block_size + p % m->block_size;
@@ -296,7 +305,7 @@ int pa_bm_take_copies(pa_block_manager* m, int64_t* pairs, int capacity) {
   if (!m || capacity < 0 || (capacity > 0 && !pairs)) return -1;
   const int n = (int)m->pending_copies.size() / 2;
   if (n > capacity) return -n;  // too small: nothing taken
-  std::memcpy(pairs, m->pending_copies.data(), sizeof(int64_t) * 2 * n);
+  if (n > 0) std::memcpy(pairs, m->pending_copies.data(), sizeof(int64_t) * 2 * n);
   m->pending_copies.clear();
   return n;
 }

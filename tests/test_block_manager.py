@@ -270,3 +270,73 @@ def test_simulated_pool_reads_back_every_sequence(seed, B):
     for sid in list(seqs):
         bm.free(sid)
     assert bm.num_free_blocks == nb
+
+
+def test_c_abi_error_returns_leave_the_manager_unchanged():
+    # every documented error of the pa_bm_* calls, through the raw C ABI
+    import ctypes
+    L = pa.lib()
+    _p = ctypes.c_void_p
+    assert L.pa_bm_create(2**27, 32, 1, ctypes.byref(_p())) == pa.PA_ERR_INVALID_ARG  # > INT32_MAX tokens
+    assert L.pa_bm_create(0, 16, 1, ctypes.byref(_p())) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_create(4, 16, 1, None) == pa.PA_ERR_INVALID_ARG
+
+    bm = pa.BlockManager(4, 16)
+    h = bm._h
+    bm.add_sequence(1, toks(20))
+    bm.fork(1, 2)
+    before = (bm.num_free_blocks, list(bm.block_table(1)), bm.ref_count(0), bm.ref_count(1))
+
+    def ptr(a):
+        return a.ctypes.data_as(_p)
+
+    small = toks(16)
+    cached = ctypes.c_int(-5)
+    assert L.pa_bm_add_sequence(h, 1, ptr(small), 16, ctypes.byref(cached)) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_add_sequence(h, 3, ptr(small), -1, None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_add_sequence(h, 3, None, 1, None) == pa.PA_ERR_INVALID_ARG
+    big = toks(5 * 16)  # needs more blocks than the pool has
+    assert L.pa_bm_add_sequence(h, 3, ptr(big), big.size, None) == pa.PA_ERR_OUT_OF_RANGE
+    # a count whose block total overflows int is refused before any token is read
+    assert L.pa_bm_add_sequence(h, 3, ptr(small), 2**31 - 1, None) == pa.PA_ERR_OUT_OF_RANGE
+    assert cached.value == -5 and bm.num_tokens(3) == -1
+
+    assert L.pa_bm_append(h, 9, ptr(small), 1) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_append(h, 1, ptr(small), -1) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_append(h, 1, None, 1) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_append(h, 1, ptr(small), 2**31 - 1) == pa.PA_ERR_OUT_OF_RANGE
+    assert bm.num_tokens(1) == 20
+
+    assert L.pa_bm_fork(h, 9, 5) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_fork(h, 1, 2) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_free(h, 9) == pa.PA_ERR_INVALID_ARG
+
+    n = ctypes.c_int(0)
+    out = np.full(1, 77, dtype=np.int32)
+    assert L.pa_bm_block_table(h, 1, ptr(out), 1, ctypes.byref(n)) == pa.PA_ERR_WORKSPACE
+    assert n.value == 2 and out[0] == 77
+    assert L.pa_bm_block_table(h, 9, ptr(out), 1, None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_block_table(h, 1, None, 2, None) == pa.PA_ERR_INVALID_ARG
+
+    slots = np.full(16, -9, dtype=np.int64)
+    # past the tokens held but inside the last block: allowed
+    assert L.pa_bm_slots(h, 1, 20, 12, ptr(slots)) == pa.PA_OK
+    assert list(slots[:12]) == list(range(20, 32)) and slots[12] == -9  # table [0, 1]
+    slots[:] = -9
+    assert L.pa_bm_slots(h, 1, 25, 8, ptr(slots)) == pa.PA_ERR_OUT_OF_RANGE  # past block 2
+    assert np.all(slots == -9)
+    assert L.pa_bm_slots(h, 1, 2**31 - 2, 5, ptr(slots)) == pa.PA_ERR_OUT_OF_RANGE  # no overflow
+    assert L.pa_bm_slots(h, 1, -1, 1, ptr(slots)) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_bm_slots(h, 9, 0, 1, ptr(slots)) == pa.PA_ERR_INVALID_ARG
+
+    bm.append(2, toks(1, 500))  # copy-on-write of the shared partial block: one pair pending
+    pairs = np.zeros((1, 2), dtype=np.int64)
+    assert L.pa_bm_take_copies(h, ptr(pairs), 0) == -1  # too small: nothing taken
+    assert L.pa_bm_take_copies(h, None, 1) == -1
+    assert L.pa_bm_take_copies(h, ptr(pairs), 1) == 1 and list(pairs[0]) == [1, 2]
+
+    assert bm.ref_count(-1) == -1 and bm.ref_count(4) == -1 and bm.num_tokens(9) == -1
+    assert L.pa_bm_num_free_blocks(None) == -1
+    # sequence 1 saw only refused calls
+    assert list(bm.block_table(1)) == before[1] and bm.num_tokens(1) == 20
+    assert bm.ref_count(0) == 2 and bm.ref_count(1) == 1 and bm.num_free_blocks == 1
