@@ -130,11 +130,22 @@ def _dtype_code(t: torch.Tensor, allow_fp8: bool = False) -> int:
                      + (" or uint8 (E4M3 codes)" if allow_fp8 else ""))
 
 
+def _check_device(t, name: str) -> None:
+    """The library launches on the calling thread's current device, so a CUDA
+    tensor argument must live there (another device's pointer would reach
+    the kernel as a foreign address)."""
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current device is cuda:{cur}; "
+                         "call under torch.cuda.device(...) of the tensors' device")
+
+
 def _ptr(t, name: str, dtype=None, ndim=None) -> Optional[int]:
     if t is None:
         return None
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    _check_device(t, name)
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -284,6 +295,8 @@ def _pool_ptr(t, name):
         raise ValueError(f"{name} must be a contiguous tensor")
     if not (t.is_cuda or t.is_pinned()):
         raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if t.is_cuda:
+        _check_device(t, name)
     return t.data_ptr()
 
 
