@@ -143,11 +143,22 @@ int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int ma
   return (p / block_size) * block_size;
 }
 
+// A caller's partition length rounded up to whole blocks; lengths above 2^30
+// tokens are clamped there first (any partition longer than every sequence
+// means one partition), so the rounding cannot overflow.
+int round_partition_tokens(int requested, int block_size) {
+  const long long r = requested > (1 << 30) ? (1 << 30) : requested;
+  return (int)(((r + block_size - 1) / block_size) * block_size);
+}
+
 int partition_tokens_for(int requested, int num_seqs, int num_kv_heads, int block_size,
                          int max_seq_len) {
-  if (requested > 0) return ((requested + block_size - 1) / block_size) * block_size;
+  if (requested > 0) return round_partition_tokens(requested, block_size);
   return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_seq_len);
 }
+
+// Partitions of a sequence of `len` tokens (at least one).
+long long num_partitions(int len, int pt) { return len == 0 ? 1 : ((long long)len + pt - 1) / pt; }
 
 template <class Tiles, int BS, int NT>
 pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
@@ -267,7 +278,7 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
 // short items (the last item of a worker bounds how long it idles at the end).
 int mixed_partition_tokens(int requested, int num_decode, int num_kv_heads, int block_size,
                            int max_dec_len) {
-  if (requested > 0) return ((requested + block_size - 1) / block_size) * block_size;
+  if (requested > 0) return round_partition_tokens(requested, block_size);
   const int p = auto_partition_tokens(num_decode, num_kv_heads, block_size, max_dec_len);
   return p > 1024 ? 1024 : p;
 }
@@ -482,7 +493,7 @@ pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_hea
     return PA_ERR_INVALID_ARG;
   const int pt = partition_tokens_for(partition_tokens, num_seqs, num_kv_heads, block_size,
                                       max_seq_len);
-  const long long parts = max_seq_len == 0 ? 1 : ((long long)max_seq_len + pt - 1) / pt;
+  const long long parts = num_partitions(max_seq_len, pt);
   if (parts <= 1) {
     *bytes = 0;
     return PA_OK;
@@ -540,8 +551,9 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
 
   const int pt = partition_tokens_for(partition_tokens, num_seqs, num_kv_heads, block_size,
                                       max_seq_len);
-  const int num_parts = max_seq_len == 0 ? 1 : (max_seq_len + pt - 1) / pt;
-  if (num_parts > 65535) return PA_ERR_INVALID_ARG;
+  const long long parts = num_partitions(max_seq_len, pt);
+  if (parts > 65535) return PA_ERR_INVALID_ARG;
+  const int num_parts = (int)parts;
   size_t need = 0;
   pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                            max_seq_len, partition_tokens, &need);
@@ -618,7 +630,7 @@ pa_status pa_append_decode(void* out, const void* query, const void* new_key,
                            int max_blocks_per_seq, int max_ctx_len, int partition_tokens,
                            float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
                            pa_stream_t stream) {
-  if (max_ctx_len < 0) return PA_ERR_INVALID_ARG;
+  if (max_ctx_len < 0 || max_ctx_len == INT_MAX) return PA_ERR_INVALID_ARG;  // decodes ctx + 1
   const AppendArgs app{new_key, new_value, slot_mapping};
   return decode_impl(out, query, key_cache, value_cache, block_tables, ctx_lens, num_seqs,
                      num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
@@ -772,13 +784,14 @@ pa_status pa_mixed_workspace_size(int num_decode_seqs, int num_q_heads, int num_
                                   int head_dim, int block_size, int max_ctx_len,
                                   int partition_tokens, size_t* bytes) {
   if (!bytes || num_decode_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-      block_size <= 0 || max_ctx_len < 0 || partition_tokens < 0)
+      block_size <= 0 || max_ctx_len < 0 || max_ctx_len == INT_MAX || partition_tokens < 0)
     return PA_ERR_INVALID_ARG;
   const int max_dec_len = max_ctx_len + 1;
   const int pt = mixed_partition_tokens(partition_tokens, num_decode_seqs > 0 ? num_decode_seqs : 1,
                                         num_kv_heads, block_size, max_dec_len);
+  // pt >= 1, so the count fits an int
   *bytes = mixed_workspace_bytes(num_decode_seqs, num_q_heads, head_dim,
-                                 (max_dec_len + pt - 1) / pt);
+                                 (int)num_partitions(max_dec_len, pt));
   return PA_OK;
 }
 
@@ -791,7 +804,8 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
                              float scale, pa_dtype dtype, void* workspace,
                              size_t workspace_bytes, pa_stream_t stream) {
   if (num_seqs < 0 || num_decode_seqs < 0 || num_decode_seqs > num_seqs ||
-      total_q < num_decode_seqs || max_q_len < 0 || max_ctx_len < 0 || num_q_heads <= 0 ||
+      total_q < num_decode_seqs || max_q_len < 0 || max_ctx_len < 0 || max_ctx_len == INT_MAX ||
+      num_q_heads <= 0 ||
       num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0 ||
       !valid_dtype(dtype) || !std::isfinite(scale))
     return PA_ERR_INVALID_ARG;
@@ -817,7 +831,7 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
   const int max_dec_len = max_ctx_len + 1;
   const int pt = mixed_partition_tokens(partition_tokens, num_decode > 0 ? num_decode : 1,
                                         num_kv_heads, block_size, max_dec_len);
-  const int num_parts = (max_dec_len + pt - 1) / pt;
+  const int num_parts = (int)num_partitions(max_dec_len, pt);
   const size_t need = mixed_workspace_bytes(num_decode, num_q_heads, head_dim, num_parts);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return PA_ERR_WORKSPACE;
   // prefill chunks: 256-row tiles per (chunk, query head)

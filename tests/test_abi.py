@@ -73,6 +73,12 @@ def test_workspace_size_is_host_only(lib):
     # would take 2048 for this batch)
     assert pa.pa_decode_partition_tokens(256, 8, 16, 4096) == 2048
     assert pa.pa_mixed_workspace_size(256, 32, 8, 128, 16, 4095) == 512 + 256 * 32 * 4 * 130 * 4
+    # a requested partition longer than every sequence is one partition (its
+    # rounding to whole blocks does not overflow)
+    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 5000, partition_tokens=2**31 - 1) == 0
+    assert pa.pa_mixed_workspace_size(4, 8, 2, 128, 16, 100, partition_tokens=2**31 - 1) == 512
+    with pytest.raises(pa.PAError):
+        pa.pa_mixed_workspace_size(4, 8, 2, 128, 16, 2**31 - 1)  # decode rows see ctx + 1
 
 
 P = ctypes.c_void_p
@@ -99,6 +105,8 @@ def test_decode_rejects_bad_arguments(lib):
     assert call(d=96) == pa.PA_ERR_UNSUPPORTED
     assert call(hq=34, hkv=1) == pa.PA_ERR_UNSUPPORTED          # group > 16
     assert call(maxl=128, pt=16) == pa.PA_ERR_WORKSPACE         # 8 partitions, no workspace
+    # a length near INT_MAX: over 65535 partitions, refused without overflowing
+    assert call(maxl=2**31 - 10, mb=2**27) == pa.PA_ERR_INVALID_ARG
     assert call(S=0) == pa.PA_OK                                # empty batch: nothing to do
 
 
@@ -136,6 +144,7 @@ def test_mixed_rejects_bad_arguments(lib):
     assert call(tq=3) == pa.PA_ERR_INVALID_ARG                  # fewer rows than decode seqs
     assert call(cu=None) == pa.PA_ERR_INVALID_ARG
     assert call(mc=16 * 16) == pa.PA_ERR_INVALID_ARG            # ctx + 1 does not fit the table
+    assert call(mc=2**31 - 1, mb=2**27) == pa.PA_ERR_INVALID_ARG  # ctx + 1 is not an int
     assert call(hq=3, hkv=2) == pa.PA_ERR_INVALID_ARG
     assert call(q=P(0x100004)) == pa.PA_ERR_INVALID_ARG         # misaligned
     assert call(d=64) == pa.PA_ERR_UNSUPPORTED
@@ -162,6 +171,7 @@ def test_append_decode_rejects_bad_arguments(lib):
     assert call(nv=P(0x100008)) == pa.PA_ERR_INVALID_ARG          # misaligned
     assert call(mc=8 * 16) == pa.PA_ERR_INVALID_ARG               # ctx + 1 does not fit
     assert call(mc=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(mc=2**31 - 1, mb=2**27) == pa.PA_ERR_INVALID_ARG  # ctx + 1 is not an int
     assert call(dt=pa.PA_FP8_E4M3) == pa.PA_ERR_INVALID_ARG       # fp16 / bf16 only
     assert call(bs=8, mb=64) == pa.PA_ERR_UNSUPPORTED
     assert call(S=0) == pa.PA_OK
