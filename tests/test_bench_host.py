@@ -10,6 +10,7 @@ import torch
 
 import synth
 
+
 def test_peaks_are_the_measured_ones(tmp_path, monkeypatch):
     import bench
     # the measured copy bandwidth and bf16 GEMM burst figure when the peaks
