@@ -4,7 +4,6 @@ in-range domain, saturation / tie cases, and round trips."""
 import math
 
 import numpy as np
-import pytest
 import torch
 
 import oracle
