@@ -29,7 +29,11 @@ __all__ = ["e4m3_value", "E4M3_TABLE", "e4m3_encode", "quantize", "paged_decode_
 
 
 def e4m3_value(code: int) -> float:
-    """The real number an E4M3 code stands for (NaN for S.1111.111)."""
+    """The real number an E4M3 code stands for (NaN for S.1111.111).
+
+    The FP8 cache of "PagedAttention: KV cache as virtual memory", "Deep dive"
+    names no format; this is the OCP E4M3 encoding read in the module header.
+    """
     code = int(code) & 0xFF
     s = -1.0 if code & 0x80 else 1.0
     e = (code >> 3) & 0xF
@@ -49,7 +53,12 @@ _MAX = float(_POS_VALUES[-1])  # 448
 
 
 def e4m3_encode(x) -> np.ndarray:
-    """Nearest E4M3 code of each float (ties to the even code, saturating)."""
+    """Nearest E4M3 code of each float (ties to the even code, saturating).
+
+    Writing into the FP8 cache of "PagedAttention: KV cache as virtual
+    memory", "Deep dive"; the rounding rule is the reading in the module
+    header (the pages fix none).
+    """
     x = np.asarray(x, dtype=np.float64)
     out = np.empty(x.shape, dtype=np.uint8)
     flat_x = x.reshape(-1)
@@ -75,7 +84,12 @@ def e4m3_encode(x) -> np.ndarray:
 
 def quantize(x, scale: float) -> np.ndarray:
     """Codes of values x (any float array, exact in fp32) under a per-cache scale:
-    fp32 division, then e4m3_encode."""
+    fp32 division, then e4m3_encode.
+
+    The per-cache scale is the module header's reading of the FP8 cache of
+    "PagedAttention: KV cache as virtual memory", "Deep dive" and
+    "Interviewer follow-ups".
+    """
     q = np.asarray(x, dtype=np.float32) / np.float32(scale)
     return e4m3_encode(q.astype(np.float32))
 
@@ -83,7 +97,13 @@ def quantize(x, scale: float) -> np.ndarray:
 def paged_decode_fp8(query, key_codes, value_codes, block_tables, seq_lens, scale, k_scale,
                      v_scale, num_kv_heads):
     """Paged decode over FP8 caches: the codes stand for code_value * scale;
-    attention is then exactly the fp64 paged decode of those values."""
+    attention is then exactly the fp64 paged decode of those values.
+
+    "PagedAttention: KV cache as virtual memory", "Interviewer follow-ups"
+    (an FP8 KV cache halves the bytes per block; attention itself is
+    unchanged), with the decode of "vLLM PagedAttention Deep Dive",
+    "PagedAttention Mechanism".
+    """
     kc = E4M3_TABLE[np.asarray(key_codes, dtype=np.uint8)] * float(np.float32(k_scale))
     vc = E4M3_TABLE[np.asarray(value_codes, dtype=np.uint8)] * float(np.float32(v_scale))
     return paged_decode(query, kc, vc, block_tables, seq_lens, scale, num_kv_heads)

@@ -220,6 +220,10 @@ def partial_attention(q, K, V, scale):
 
     m = max_j z_j, l = sum_j exp(z_j - m), acc = sum_j exp(z_j - m) V_j with
     z = scale * K q.  An empty range gives (-inf, 0, 0).
+
+    The pages do not split the key range; this is the standard attention of
+    [Deep Dive] "PagedAttention Mechanism" kept unnormalised over one range,
+    so that combine_partials can recover it exactly.
     """
     q = np.asarray(q, dtype=np.float64)
     if K.shape[0] == 0:
@@ -236,7 +240,9 @@ def combine_partials(states):
     With M = max_p m_p: o = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p.
     This is exactly softmax attention over the union of the key ranges (the
     rescaling cancels), which the split-KV tests check against the unsplit
-    result.  No keys at all gives zeros.
+    result.  No keys at all gives zeros.  Cited passage: the standard
+    attention of [Deep Dive] "PagedAttention Mechanism"; the combine is an
+    identity of that softmax, not a step the pages describe.
     """
     ms = np.array([s[0] for s in states], dtype=np.float64)
     if ms.size == 0 or np.all(np.isneginf(ms)):
