@@ -69,7 +69,8 @@ typedef struct CUstream_st *pa_stream_t; /* same type as cudaStream_t */
 /* Human-readable name of a pa_status value.  Never NULL. */
 const char *pa_status_string(int status);
 
-/* Library ABI version, (major << 16) | minor. */
+/* Library ABI version, (major << 16) | minor.  A library service (no
+ * counterpart on the pages). */
 int pa_version(void);
 
 /*
@@ -113,8 +114,12 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *key_cac
                                pa_dtype dtype, pa_stream_t stream);
 
 /*
- * pa_append — pa_slot_mapping and pa_reshape_and_cache fused into one launch:
- * each new token's slot is computed from block_tables / cu_q_lens / ctx_lens
+ * pa_append — pa_slot_mapping and pa_reshape_and_cache fused into one launch.
+ *   "PagedAttention: KV cache as virtual memory", "Deep dive" (new tokens go
+ *   to the end of the sequence, a block being taken when the last one fills)
+ *   and "vLLM PagedAttention Deep Dive", "Mechanics of Chunked Prefill"
+ *   (a chunk's K/V accumulate in paged blocks).
+ * Each new token's slot is computed from block_tables / cu_q_lens / ctx_lens
  * (same rule as pa_slot_mapping) and its K and V rows are written there (bit
  * copy).  slot_mapping (int64[num_tokens]) receives the slots when non-NULL.
  * Same layouts and argument meanings as the two calls it fuses; a position
@@ -188,15 +193,20 @@ pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, uint8_t *
 /*
  * pa_decode_partition_tokens — the split-KV partition length pa_decode uses
  * for these sizes when called with partition_tokens == 0 (a multiple of
- * block_size).  Host-only; touches no GPU.
+ * block_size).  Host-only; touches no GPU.  The pages do not split a
+ * sequence; partitioning is this library's way to spread a decode over the
+ * GPU, and the combine is exact (see pa_decode).  Returns 0 for a
+ * non-positive count or size or a negative max_seq_len.
  */
 int pa_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_seq_len);
 
 /*
  * pa_decode_workspace_size — bytes of scratch pa_decode needs for its split-KV
- * partial results.  Host-only; touches no GPU.  partition_tokens as in
- * pa_decode (0 = automatic).  Writes 0 when no sequence can span more than one
- * partition.
+ * partial results (a library service; the pages have no workspace).
+ * Host-only; touches no GPU.  partition_tokens as in pa_decode (0 =
+ * automatic).  Writes 0 when no sequence can span more than one partition.
+ * PA_ERR_INVALID_ARG for a null `bytes`, a negative num_seqs, max_seq_len or
+ * partition_tokens, or a non-positive head count, head_dim or block_size.
  */
 pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                    int block_size, int max_seq_len, int partition_tokens,
@@ -266,7 +276,10 @@ pa_status pa_append_decode(void *out, const void *query, const void *new_key,
 
 /*
  * pa_decode_fp8 — pa_decode over FP8 (E4M3) caches (see pa_reshape_and_cache_fp8
- * for the encoding).  Attention is computed over the values code * k_scale and
+ * for the encoding).
+ *   "PagedAttention: KV cache as virtual memory", "Interviewer follow-ups"
+ *   (an FP8 KV cache halves the bytes per block; attention is unchanged).
+ * Attention is computed over the values code * k_scale and
  * code * v_scale; the query and output are fp16 or bf16 (`dtype`).  The
  * products run on fp16 tensor-core MMAs with fp32 accumulation: E4M3 codes
  * are exact in fp16, the query is rounded to fp16 (exact for |q| in fp16's
@@ -482,8 +495,8 @@ int pa_bm_ref_count(const pa_block_manager *bm, int block);
 int pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id);
 
 /*
- * pa_get_device_error — synchronise `stream`, then read and clear the device
- * error word of the current device (a bitwise OR of PA_DEVERR_* since the
+ * pa_get_device_error — a library service (no counterpart on the pages):
+ * synchronise `stream`, then read and clear the device error word of the current device (a bitwise OR of PA_DEVERR_* since the
  * last read).  Returns PA_ERR_OUT_OF_RANGE when the word was non-zero.
  */
 pa_status pa_get_device_error(unsigned int *error_word, pa_stream_t stream);
