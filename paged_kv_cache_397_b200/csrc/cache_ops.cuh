@@ -115,7 +115,9 @@ __global__ void append_kernel(const uint4* __restrict__ key, const uint4* __rest
   value_cache[dst] = vv;
 }
 
-// One thread per 16-byte chunk of one (token, kv head) row of K and of V.
+// One thread per 16-byte chunk of one (token, kv head) row of K and of V
+// ("PagedAttention: KV cache as virtual memory", "Deep dive": a new token's
+// K/V go into the next free slot of its sequence's last block).
 template <int D>
 __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
                                          const uint4* __restrict__ value,
@@ -201,6 +203,9 @@ __global__ void reshape_and_cache_fp8_kernel(const T* __restrict__ key, const T*
   }
 }
 
+// Copy-on-write block copies ("PagedAttention: Why Static Batching Wastes
+// Your KV Cache", "How does copy-on-write eliminate duplicate prompt KV
+// cache?": the diverging sequence gets its own copy of just that block).
 // One CTA per (pair, K-or-V); each thread moves kPerThread 16-byte chunks,
 // all loads issued before the stores.
 template <int kPerThread>
@@ -231,7 +236,9 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Block copies between two pools (swap out to / in from host memory).  One
+// Block copies between two pools (swap out to / in from host memory;
+// "PagedAttention: Why Static Batching Wastes Your KV Cache", "What happens
+// when the GPU runs out of KV blocks?").  One
 // CTA per (pair, K-or-V); either pool may be pinned host memory mapped into
 // the GPU's address space, so the loads or the stores cross PCIe / C2C; all
 // of a thread's loads are issued before its stores to keep many in flight.
