@@ -496,8 +496,13 @@ int pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id);
 
 /*
  * pa_get_device_error — a library service (no counterpart on the pages):
- * synchronise `stream`, then read and clear the device error word of the current device (a bitwise OR of PA_DEVERR_* since the
- * last read).  Returns PA_ERR_OUT_OF_RANGE when the word was non-zero.
+ * synchronise `stream`, then read and clear the device error word of the
+ * current device (a bitwise OR of PA_DEVERR_* since the last read).  Returns
+ * PA_ERR_OUT_OF_RANGE when the word was non-zero, PA_ERR_CUDA if the
+ * synchronisation or the copies fail.  The read and the clear are two copies:
+ * a kernel still running on another stream can set a bit between them and
+ * that bit is lost, so synchronise every stream that launched library
+ * kernels before calling this.
  */
 pa_status pa_get_device_error(unsigned int *error_word, pa_stream_t stream);
 

@@ -75,16 +75,16 @@ static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORK
 
 constexpr int kMaxDevices = 64;
 int sm_count() {
-  static int cached[kMaxDevices] = {};
+  static std::atomic<int> cached[kMaxDevices];  // zero-initialised (static storage)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);  // every thread stores the same value
   }
-  return cached[dev];
+  return n;
 }
 
 // One-time per (kernel, device) launch configuration: the dynamic shared
