@@ -1,7 +1,10 @@
 """pa_prefill_chunk (tcgen05) against the fp64 oracle: ragged chunks and
 contexts across several 128-row / 128-key tiles, both block sizes and both
-16-bit types, NaN in unused slots, and the full-size 8 x 512-token chunk
-workload on sampled rows."""
+16-bit types, NaN in unused slots, the full-size 8 x 512-token chunk
+workload on sampled rows, and bit-identical output under a relabelling of the
+physical blocks, with and without the key-range split of the last wave."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -110,3 +113,45 @@ def test_split_tail_is_deterministic():
     runs = [run_prefill(p, split_tail=True) for _ in range(3)]
     for r in runs[1:]:
         assert torch.equal(r.view(torch.int16), runs[0].view(torch.int16))
+
+
+def _relabelled(p, seed):
+    """The same chunk batch with every physical block moved to a new id
+    (block b -> perm[b]); the tables follow, so the logical K/V are unchanged."""
+    perm = torch.randperm(p.num_blocks, generator=torch.Generator().manual_seed(seed))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(p.num_blocks)
+    bt = p.block_tables.clone()
+    bt[bt >= 0] = perm[bt[bt >= 0].long()].to(bt.dtype)
+    return dataclasses.replace(p, key_cache=p.key_cache[inv].contiguous(),
+                               value_cache=p.value_cache[inv].contiguous(), block_tables=bt)
+
+
+# Work units = 256-row tiles x query heads x sequences; on 148 SMs the units of
+# the last wave are cut along the key range into k parts: 16 units -> k = 4,
+# 40 units -> k = 3, 64 units -> k = 2 (k minimises ceil(units * k / 148) / k).
+RELABEL_CASES = {
+    "split4": dict(hq=4, hkv=2, ctx_lens=[700, 3], q_lens=[300, 257]),
+    "split3": dict(hq=4, hkv=4, ctx_lens=[0, 5, 40, 900, 129], q_lens=[1, 130, 7, 300, 256]),
+    "split2": dict(hq=8, hkv=2, ctx_lens=[1000, 17, 260, 64], q_lens=[511, 300, 2, 129]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(RELABEL_CASES))
+@pytest.mark.parametrize("B", [16, 32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_prefill_bit_identical_under_block_relabelling(case, B, dtype):
+    # The result may depend only on logical positions, never on where the
+    # blocks sit in the pool ("vLLM PagedAttention Deep Dive", "PagedAttention
+    # Mechanism"): with and without the key-range split of the last wave.
+    p = synth.chunked_prefill(seed=31 + B, block_size=B, dtype=dtype, d=128,
+                              **RELABEL_CASES[case])
+    moved = _relabelled(p, seed=5 + B)
+    for split_tail in (True, False):
+        a = run_prefill(p, split_tail)
+        b = run_prefill(moved, split_tail)
+        assert torch.isfinite(a.float()).all()
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (case, split_tail)
+    oracle_scatter(p)
+    ref, _ = reference(p)
+    assert max_err(a, ref) <= TOL[dtype]

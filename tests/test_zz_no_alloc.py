@@ -4,10 +4,16 @@ Some callers of this library may not call cudaMalloc — a plugin inside an
 inference runtime that owns and budgets every byte of device memory, or a
 serving loop that must not allocate after start-up.  This entry point keeps
 pa_decode's split-KV scratch in the library's own per-device array instead of
-a caller workspace.  The test calls it through the C ABI (ctypes) twice in a
-row, on different inputs, and checks each result against pa_decode with a
-caller-provided workspace, within the decode tolerance; it also checks that a
-request needing more scratch than the array holds is refused up front.
+a caller workspace.
+
+The test calls it through the C ABI (ctypes) twice in a row, on two different
+batches whose partial results have different shapes (sequence count,
+partitions per sequence, hence the row stride inside the shared array), so a
+reduce that read partials left over from the first call would be caught.
+Each result must equal pa_decode with a caller-provided workspace and the same
+partition length bit for bit (the same kernels run on the same inputs), and
+must match the fp64 oracle within the decode tolerance.  A request needing more
+scratch than the array holds must be refused up front.
 
 The file is named to be collected last, so a run that stops at the first
 failure has already run every other test; it passes alone in a fresh process
@@ -20,7 +26,7 @@ import torch
 
 import paged_kv_cache_397_b200 as pa
 import synth
-from helpers import TOL, dev, to_dev
+from helpers import TOL, decode_reference, dev, max_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -36,28 +42,37 @@ def _c_call(out, q, kc, vc, bt, lens, max_len, scale, partition_tokens):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
+# Two batches in a row: 8 sequences x 17 partitions of 256 tokens, then 5
+# sequences x 16 partitions of 128 tokens (a different partial-row layout).
+CALLS = [
+    dict(seed=42, lens=[1, 16, 17, 300, 1000, 2049, 3000, 4097], pt=256),
+    dict(seed=43, lens=[2000, 50, 1, 700, 1500], pt=128),
+]
+
+
 def test_static_workspace_matches_pa_decode_on_two_calls():
     pa.pa_get_device_error()
-    lens = [1, 16, 17, 300, 1000, 2049, 3000, 4097]
-    w = synth.random_decode(42, lens, dtype=torch.bfloat16, block_size=16, hq=32, hkv=8, d=128,
-                            append=False)
-    pt = 256  # several partitions per long sequence, so the scratch is really used
-    need = pa.pa_decode_workspace_size(w.num_seqs, 32, 8, 128, 16, max(lens), pt)
-    assert 0 < need <= pa.PA_STATIC_WORKSPACE_BYTES
-    kc, vc, bt = to_dev(w.key_cache), to_dev(w.value_cache), to_dev(w.block_tables)
-    ld = to_dev(torch.tensor(lens, dtype=torch.int32))
-    g = torch.Generator().manual_seed(7)
-    for call in range(2):
-        q = w.query if call == 0 else torch.randn(w.query.shape, generator=g).to(w.dtype)
-        q = to_dev(q)
+    parts_seen = set()
+    for c in CALLS:
+        lens, pt = c["lens"], c["pt"]
+        w = synth.random_decode(c["seed"], lens, dtype=torch.bfloat16, block_size=16, hq=32,
+                                hkv=8, d=128, append=False)
+        need = pa.pa_decode_workspace_size(w.num_seqs, 32, 8, 128, 16, max(lens), pt)
+        assert 0 < need <= pa.PA_STATIC_WORKSPACE_BYTES
+        parts_seen.add((w.num_seqs, -(-max(lens) // pt)))
+        kc, vc, bt = to_dev(w.key_cache), to_dev(w.value_cache), to_dev(w.block_tables)
+        ld = to_dev(torch.tensor(lens, dtype=torch.int32))
+        q = to_dev(w.query)
         want = torch.empty_like(q)
         pa.pa_decode(want, q, kc, vc, bt, ld, max(lens), w.scale, partition_tokens=pt)
         got = torch.full_like(q, float("nan"))
         st = _c_call(got, q, kc, vc, bt, ld, max(lens), w.scale, pt)
         assert st == pa.PA_OK, pa.pa_status_string(st)
         torch.cuda.synchronize()
-        assert torch.isfinite(got.float()).all()
-        assert (got.float() - want.float()).abs().max().item() <= TOL[w.dtype]
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+        ref = decode_reference(w, lens, list(range(w.num_seqs)))
+        assert max_err(got.cpu(), ref) <= TOL[w.dtype]
+    assert len(parts_seen) == 2  # the two calls really lay the scratch out differently
     assert pa.pa_get_device_error() == 0
 
 
