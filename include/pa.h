@@ -193,7 +193,9 @@ pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, uint8_t *
 /*
  * pa_decode_partition_tokens — the split-KV partition length pa_decode uses
  * for these sizes when called with partition_tokens == 0 (a multiple of
- * block_size).  Host-only; touches no GPU.  The pages do not split a
+ * block_size).  Host-only: it launches nothing and reads only the SM count of
+ * the current device (148, a B200's count, when no device is visible), so the
+ * choice depends on sizes and the GPU model, never on data.  The pages do not split a
  * sequence; partitioning is this library's way to spread a decode over the
  * GPU, and the combine is exact (see pa_decode).  Returns 0 for a
  * non-positive count or size or a negative max_seq_len.
@@ -203,7 +205,8 @@ int pa_decode_partition_tokens(int num_seqs, int num_kv_heads, int block_size, i
 /*
  * pa_decode_workspace_size — bytes of scratch pa_decode needs for its split-KV
  * partial results (a library service; the pages have no workspace).
- * Host-only; touches no GPU.  partition_tokens as in pa_decode (0 =
+ * Host-only (launches nothing; the automatic partition length reads the
+ * current device's SM count).  partition_tokens as in pa_decode (0 =
  * automatic).  Writes 0 when no sequence can span more than one partition.
  * PA_ERR_INVALID_ARG for a null `bytes`, a negative num_seqs, max_seq_len or
  * partition_tokens, or a non-positive head count, head_dim or block_size.
@@ -311,7 +314,10 @@ pa_status pa_decode_fp8(void *out, const void *query, const uint8_t *key_cache,
  *     PA_STATIC_WORKSPACE_BYTES return PA_ERR_WORKSPACE before any launch.
  *   - The first call on a device (with that device current) resolves the
  *     array's device address with cudaGetSymbolAddress and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  The cached address lives as
+ *     long as the device's primary context: do not reset the device
+ *     (cudaDeviceReset) between calls, or the next call would hand the
+ *     kernels a stale address.
  *   - Every call on a device shares the one array, and it keeps the last
  *     call's contents.  The decode kernels write every partial result before
  *     they read it, so nothing needs clearing; but calls that overlap on the
@@ -493,6 +499,22 @@ int pa_bm_take_copies(pa_block_manager *bm, int64_t *pairs, int capacity);
 int pa_bm_num_free_blocks(const pa_block_manager *bm);
 int pa_bm_ref_count(const pa_block_manager *bm, int block);
 int pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id);
+
+/*
+ * pa_selftest_wait_timeout — a library service (no counterpart on the
+ * pages): exercises the bounded-wait failure path on the GPU without
+ * breaking anything.  One CTA of two roles waits on barriers that nothing
+ * arrives on: role 0 gives up after limit_ns nanoseconds and raises the
+ * CTA's abort word; role 1, which has the kernels' normal 4 s limit, sees the
+ * word and gives up right after.  PA_DEVERR_WAIT_TIMEOUT is then set in the
+ * device error word (read it with pa_get_device_error) and the context stays
+ * usable.  Every kernel of this library handles a lost arrival the same way:
+ * the first wait that runs out ends the whole CTA.
+ *   limit_ns   1,000 .. 100,000,000 (1 us .. 100 ms), else PA_ERR_INVALID_ARG
+ *   waited_ns  out  uint64[2] device memory (8-byte aligned) receiving each
+ *              role's waiting time in ns, or NULL
+ */
+pa_status pa_selftest_wait_timeout(uint64_t limit_ns, uint64_t *waited_ns, pa_stream_t stream);
 
 /*
  * pa_get_device_error — a library service (no counterpart on the pages):

@@ -26,7 +26,7 @@ __all__ = [
     "pa_slot_mapping", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_partition_tokens",
     "pa_decode_workspace_size", "pa_decode", "pa_decode_static_workspace",
     "pa_prefill_workspace_size", "pa_prefill_chunk",
-    "pa_get_device_error", "PA_STATIC_WORKSPACE_BYTES",
+    "pa_get_device_error", "pa_selftest_wait_timeout", "PA_STATIC_WORKSPACE_BYTES",
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
     "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_append",
@@ -71,6 +71,7 @@ _SIGS = {
     "pa_mixed_attention": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i,
                                 _i, _i, _i, _i, _f, _i, _p, _sz, _p]),
     "pa_get_device_error": (_i, [ctypes.POINTER(ctypes.c_uint), _p]),
+    "pa_selftest_wait_timeout": (_i, [ctypes.c_uint64, _p, _p]),
     "pa_bm_create": (_i, [_i, _i, _i, ctypes.POINTER(_p)]),
     "pa_bm_destroy": (None, [_p]),
     "pa_bm_add_sequence": (_i, [_p, ctypes.c_int64, _p, _i, ctypes.POINTER(_i)]),
@@ -503,6 +504,18 @@ def pa_mixed_attention(out, query, key_cache, value_cache, block_tables, cu_q_le
         int(block_tables.shape[1]), int(partition_tokens), float(scale), _dtype_code(key_cache),
         ws_ptr, ws_bytes, _stream(stream)))
     return out
+
+
+def pa_selftest_wait_timeout(limit_ns: int, waited_ns=None, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (include/pa.h): a wait with a
+    limit of ``limit_ns`` on a barrier nothing arrives on, and a second wait
+    of the same CTA that must give up with it.  ``waited_ns``: an int64 CUDA
+    tensor of 2 elements receiving each wait's duration, or None."""
+    ptr = _ptr(waited_ns, "waited_ns", torch.int64, 1) if waited_ns is not None else None
+    if waited_ns is not None and waited_ns.numel() != 2:
+        raise ValueError("waited_ns must hold 2 elements")
+    _check("pa_selftest_wait_timeout",
+           lib().pa_selftest_wait_timeout(int(limit_ns), ptr, _stream(stream)))
 
 
 def pa_get_device_error(stream=None) -> int:

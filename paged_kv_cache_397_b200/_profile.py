@@ -4,6 +4,9 @@
     python -m paged_kv_cache_397_b200._profile decode-fp8 --seqs 64
     python -m paged_kv_cache_397_b200._profile prefill --seqs 4 [--block-size 16]
     python -m paged_kv_cache_397_b200._profile mixed --seqs 64
+    python -m paged_kv_cache_397_b200._profile decode-llama2 --seqs 16
+    python -m paged_kv_cache_397_b200._profile decode-long --seqs 2 [--block-size 16]
+    python -m paged_kv_cache_397_b200._profile decode-cow
 
 Each case builds a scaled-down copy of a bench workload (same shapes, head
 counts, length distribution and block shuffling; fewer sequences), runs the
@@ -99,9 +102,49 @@ def mixed_case(seqs: int, reps: int = 3):
     print(f"mixed case: {p.name}, decode K/V bytes {kv}, prefill causal FLOP {flops}")
 
 
+def _plain_decode(w, lens, d, reps, tables=None, caches=None):
+    kc, vc = (w.key_cache.to(d), w.value_cache.to(d)) if caches is None else caches
+    bt = (w.block_tables if tables is None else tables).to(d)
+    ld = torch.tensor(lens, dtype=torch.int32, device=d)
+    q = w.query.to(d)
+    out = torch.empty_like(q)
+    for _ in range(reps):
+        pa.pa_decode(out, q, kc, vc, bt, ld, max(lens), w.scale)
+    torch.cuda.synchronize()
+    return 2 * w.num_kv_heads * w.head_dim * w.key_cache.element_size() * sum(lens)
+
+
+def decode_llama2_case(seqs: int, reps: int = 3):
+    """The Llama-2-13B-shaped decode (fp16, 40 q = 40 kv heads) on `seqs` sequences."""
+    w = synth.llama2_13b_decode(num_seqs=seqs)
+    kv = _plain_decode(w, w.context_lens.tolist(), torch.device("cuda:0"), reps)
+    print(f"decode-llama2 case: {w.name}, K/V bytes per launch {kv}")
+
+
+def decode_long_case(seqs: int, block_size: int, reps: int = 3):
+    """The long-context split-KV decode (32768 tokens per sequence) on `seqs` sequences."""
+    w = synth.long_context_decode(num_seqs=seqs, block_size=block_size)
+    kv = _plain_decode(w, w.context_lens.tolist(), torch.device("cuda:0"), reps)
+    print(f"decode-long case: {w.name}, K/V bytes per launch {kv}")
+
+
+def decode_cow_case(reps: int = 3):
+    """The shared-prefix batch (128 sequences) after its copy-on-write and remap."""
+    w = synth.shared_prefix_cow()
+    d = torch.device("cuda:0")
+    kc, vc = w.key_cache.to(d), w.value_cache.to(d)
+    src = w.shared_blocks[w.cow_logical_block].repeat(w.num_seqs)
+    pa.pa_copy_blocks(kc, vc, torch.stack([src, w.cow_dst_blocks], 1).to(torch.int64).to(d))
+    bt = w.block_tables.clone()
+    bt[:, w.cow_logical_block] = w.cow_dst_blocks.to(torch.int32)
+    kv = _plain_decode(w, w.context_lens.tolist(), d, reps, tables=bt, caches=(kc, vc))
+    print(f"decode-cow case: {w.name}, logical K/V bytes per launch {kv}")
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode", "decode-fp8", "prefill", "mixed"])
+    ap.add_argument("case", choices=["decode", "decode-fp8", "prefill", "mixed", "decode-llama2",
+                                     "decode-long", "decode-cow"])
     ap.add_argument("--seqs", type=int, default=None)
     ap.add_argument("--block-size", type=int, default=16)
     a = ap.parse_args()
@@ -112,6 +155,12 @@ def main():
         decode_fp8_case(a.seqs or 64)
     elif a.case == "mixed":
         mixed_case(a.seqs or 64)
+    elif a.case == "decode-llama2":
+        decode_llama2_case(a.seqs or 16)
+    elif a.case == "decode-long":
+        decode_long_case(a.seqs or 2, a.block_size)
+    elif a.case == "decode-cow":
+        decode_cow_case()
     else:
         prefill_case(a.seqs or 4, a.block_size)
     if pa.pa_get_device_error():

@@ -374,7 +374,7 @@ struct DecodeShape {
   static constexpr int RING_BYTES = NS * STAGE_BYTES;
   static constexpr int MERGE_BYTES = NW * (NT * 8) * (D + 2) * 4;
   static constexpr int BODY_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + BODY_BYTES + 2 * NS * 8;
+  static constexpr int SMEM_BYTES = 1024 + BODY_BYTES + 2 * NS * 8 + 16;  // + abort word
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
   static_assert(NS % NW == 0, "ring depth vs consumer warps");
@@ -404,15 +404,19 @@ __device__ __forceinline__ int decode_parts(int nblk_seq, int part_blocks) {
 // (the last stage of an item may hold fewer), into ring positions g0, g0 + 1,
 // ... (position i uses stage i % NS and is that stage's (i / NS)-th fill).
 // Block ids are fetched once, coalesced; entries past nblk are never read.
+// Lane 0 waits, arms and loads; it returns (on lane 0) the first ring position
+// not armed, `g0` plus the item's stages unless a wait gave up (`alive`
+// false on lane 0), after which nothing more is armed or loaded.
 template <class Tiles, int BS, int NT>
-__device__ __forceinline__ bool produce_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                             const DecodeParams& p, uint8_t* ring,
-                                             uint64_t* full_bar, uint64_t* empty_bar, int s,
-                                             int kvh, int blk0, int nblk, int g0, int lane,
-                                             uint64_t policy, bool alive) {
+__device__ __forceinline__ int produce_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                            const DecodeParams& p, uint8_t* ring,
+                                            uint64_t* full_bar, uint64_t* empty_bar, int s,
+                                            int kvh, int blk0, int nblk, int g0, int lane,
+                                            uint64_t policy, bool& alive, volatile int* abort) {
   using Shape = DecodeShape<Tiles, BS, NT>;
   constexpr int NS = Shape::NS, SB = Shape::SB;
   const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+  int armed = g0;
   for (int base = 0; base < nblk; base += 32) {
     int phys = 0;
     if (base + lane < nblk) {
@@ -430,19 +434,22 @@ __device__ __forceinline__ bool produce_item(const CUtensorMap* tm_k, const CUte
       if (lane == 0) {
         const int nb = min(SB, cnt - j);  // blocks in this stage
         const int i = g0 + (base + j) / SB, st = i % NS;
-        if (i >= NS && alive) alive = mbar_wait(&empty_bar[st], ((i / NS) - 1) & 1);
-        mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
-        uint8_t* sk = ring + st * Shape::STAGE_BYTES;
+        if (i >= NS && alive) alive = mbar_wait(&empty_bar[st], ((i / NS) - 1) & 1, abort);
+        if (alive) {
+          mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
+          uint8_t* sk = ring + st * Shape::STAGE_BYTES;
 #pragma unroll
-        for (int u = 0; u < SB; ++u)
-          if (u < nb)
-            Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
-                         (ph[u] * p.num_kv_heads + kvh * Shape::HP) * BS, u, &full_bar[st],
-                         policy);
+          for (int u = 0; u < SB; ++u)
+            if (u < nb)
+              Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
+                           (ph[u] * p.num_kv_heads + kvh * Shape::HP) * BS, u, &full_bar[st],
+                           policy);
+          armed = i + 1;
+        }
       }
     }
   }
-  return alive;
+  return armed;
 }
 
 // Online softmax of one consumer warp over one ring stage (TT tokens of HP
@@ -673,7 +680,9 @@ __device__ __forceinline__ void append_new_token(const DecodeParams& p, int s, i
 // run by THREADS consecutive threads (`tid` 0 .. THREADS-1) that own the
 // 1024-byte aligned shared memory at `smem` (SMEM_BYTES - 1024 bytes).  They
 // synchronise among themselves only, on named barriers `bar_all` (all
-// THREADS) and `bar_consumers` (the NW consumer warps).
+// THREADS) and `bar_consumers` (the NW consumer warps).  A wait that gives up
+// ends the item: the producer stops loading, the consumers skip the rest, and
+// the producer drains its loads in flight before the threads leave.
 template <class Tiles, int BS, int NT>
 __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                             const DecodeParams& p, uint8_t* smem, int part,
@@ -684,6 +693,7 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Shape::BODY_BYTES);
   uint64_t* empty_bar = full_bar + NS;
+  volatile int* abort = reinterpret_cast<volatile int*>(empty_bar + NS);
   const int warp = tid >> 5, lane = tid & 31;
 
   const int L = decode_len<BS>(p, s, tid == 0 && part == 0 && kvh == 0);
@@ -698,6 +708,7 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], 1);
     }
+    *abort = 0;
     fence_barrier_init();
   }
   named_barrier(bar_all, Shape::THREADS);
@@ -718,8 +729,12 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
           p.slot_out[s] = -1;
       }
     }
-    produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s, kvh, blk0, nblk, 0,
-                                lane, l2_policy_evict_first(), true);
+    bool alive = true;
+    const int armed = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s,
+                                                  kvh, blk0, nblk, 0, lane,
+                                                  l2_policy_evict_first(), alive, abort);
+    named_barrier(bar_all, Shape::THREADS);  // the consumers are done
+    if (*abort && lane == 0) drain_ring<NS>(full_bar, armed);
     return;
   }
 
@@ -733,13 +748,15 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   float m_run[NT][2], l_run[NT][2];
   float o[D / 16][NT][4];
   reset_state<Tiles, NT>(o, m_run, l_run);
-  bool alive = true;
   const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
   // a stage may reach past the item's last block (into the next partition)
   const int L_end = min(L, (blk0 + nblk) * BS);
+  bool alive = true;
   for (int i = warp; i < nstages; i += NW) {
     const int st = i % NS;
-    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1);
+    // after a wait gave up the warp still runs through its (garbage) stages,
+    // every lane alike, so the .aligned loads and MMAs stay converged
+    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1, abort);
     consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
                                  (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane,
                                  p.group);
@@ -747,9 +764,11 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
     if (lane == 0) mbar_arrive(&empty_bar[st]);
   }
   // the merge area aliases the ring: merge_item's opening barrier waits for
-  // every consumer to finish reading it
+  // every consumer to finish reading it (after an abort a late load may still
+  // land there; the output is garbage then, and the error word says so)
   merge_item<Tiles, BS, NT>(reinterpret_cast<float*>(smem), o, m_run, l_run, p, s, kvh, part,
                             nparts == 1, tid, bar_consumers);
+  named_barrier(bar_all, Shape::THREADS);  // lets the producer see the final abort word
 }
 
 template <class Tiles, int BS, int NT>

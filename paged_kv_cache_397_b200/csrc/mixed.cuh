@@ -46,15 +46,18 @@ struct WorkerShape {
   static constexpr int BAR_OFF = MERGE_OFF + Dc::MERGE_BYTES;
   static constexpr int NBAR = 2 * Dc::NS + 2 * QD;
   static constexpr int ITEM_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int BYTES = (ITEM_OFF + (QD + 1) * 4 + 1023) / 1024 * 1024;
+  // item slots, the current item, the worker's abort word
+  static constexpr int BYTES = (ITEM_OFF + (QD + 2) * 4 + 1023) / 1024 * 1024;
 };
 
 // A persistent decode worker (THREADS = 160 threads, `tid` 0..159): takes work
 // items i = atomicAdd(queue, 1) until i >= num_items; item i is partition
 // i % max_parts of KV head (i / max_parts) % Hkv of sequence
 // i / (max_parts * Hkv).  Items past a sequence's last partition are skipped
-// by the producer.  Every wait is bounded; a consumer-side timeout ends the
-// worker (and the error word says so).
+// by the producer.  Every wait is bounded; a wait that gives up ends the
+// worker: the producer stops taking items and loading, the consumers stop at
+// the next item, and the producer drains its loads in flight before the
+// worker's threads leave (the error word says so).
 template <class Tiles, int BS, int NT>
 __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const DecodeParams& p, uint8_t* smem, int* queue,
@@ -70,6 +73,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
   uint64_t* item_empty = item_full + QD;
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + W::ITEM_OFF);
   volatile int* cur_item = item_slot + QD;
+  volatile int* abort = cur_item + 1;
   float* mg = reinterpret_cast<float*>(smem + W::MERGE_OFF);
   const int warp = tid >> 5, lane = tid & 31;
   const int per_seq = p.max_parts * p.num_kv_heads;
@@ -83,6 +87,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], 1);
     }
+    *abort = 0;
     fence_barrier_init();
   }
   named_barrier(bar_all, Shape::THREADS);
@@ -116,15 +121,19 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
       }
       const int slot = k % QD;
       if (lane == 0) {
-        if (k >= QD && alive) alive = mbar_wait(&item_empty[slot], ((k / QD) - 1) & 1);
-        item_slot[slot] = item;
+        if (k >= QD && alive) alive = mbar_wait(&item_empty[slot], ((k / QD) - 1) & 1, abort);
+        item_slot[slot] = alive ? item : -1;  // after an abort: tell the consumers to stop
         mbar_arrive(&item_full[slot]);  // release: the consumers' wait acquires item_slot
       }
-      if (item < 0) break;
-      alive = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s, kvh,
-                                          part * p.part_blocks, nblk, g, lane, policy, alive);
-      g += (nblk + Shape::SB - 1) / Shape::SB;
+      alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
+      if (item < 0 || !alive) break;
+      const int next = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s,
+                                                   kvh, part * p.part_blocks, nblk, g, lane,
+                                                   policy, alive, abort);
+      g = __shfl_sync(0xffffffffu, next, 0);  // lane 0's count (the lanes agree unless aborted)
     }
+    named_barrier(bar_all, Shape::THREADS);  // the consumers are done
+    if (*abort && lane == 0) drain_ring<NS>(full_bar, g);
     return;
   }
 
@@ -136,7 +145,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
   for (int k = 0;; ++k) {
     if (tid == 0) {
       const int slot = k % QD;
-      const bool ok = mbar_wait(&item_full[slot], (k / QD) & 1);
+      const bool ok = mbar_wait(&item_full[slot], (k / QD) & 1, abort);
       *cur_item = ok ? item_slot[slot] : -1;
       mbar_arrive(&item_empty[slot]);
     }
@@ -161,13 +170,13 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     float m_run[NT][2], l_run[NT][2];
     float o[D / 16][NT][4];
     reset_state<Tiles, NT>(o, m_run, l_run);
-    bool alive = true;
     const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
     // a stage may reach past the item's last block (into the next partition)
     const int L_end = min(L, (blk0 + nblk) * BS);
+    bool alive = true;
     for (int i = warp; i < nstages; i += NW) {
       const int gi = g + i, st = gi % NS;
-      if (alive) alive = mbar_wait(&full_bar[st], (gi / NS) & 1);
+      if (alive) alive = mbar_wait(&full_bar[st], (gi / NS) & 1, abort);
       consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
                                    (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane);
       __syncwarp();
@@ -179,6 +188,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     merge_item<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, nparts == 1, tid,
                               bar_consumers);
   }
+  named_barrier(bar_all, Shape::THREADS);  // lets the producer see the final abort word
 }
 
 template <typename T, int BS, int NT>

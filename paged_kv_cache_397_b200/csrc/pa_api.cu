@@ -131,11 +131,12 @@ pa_status static_workspace_address(void** addr) {
 }
 
 // Split-KV partition length in tokens.  Partitions are whole blocks; the aim
-// is several waves of CTAs over 148 SMs while keeping each partition long
-// enough (>= 256 tokens) that its fixed cost and its partial write stay small.
+// is several waves of CTAs over the device's SMs while keeping each partition
+// long enough (>= 256 tokens) that its fixed cost and its partial write stay
+// small.  The choice depends only on sizes and the SM count, never on data.
 int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_seq_len) {
   const long long units = (long long)num_seqs * num_kv_heads;
-  const long long target_ctas = 148LL * 3 * 8;  // ~8 waves at 3 CTAs per SM
+  const long long target_ctas = (long long)sm_count() * 3 * 8;  // ~8 waves at 3 CTAs per SM
   long long per = (long long)max_seq_len * units / target_ctas;
   int p = 256;
   while (p < 2048 && p < per) p *= 2;
@@ -330,6 +331,30 @@ pa_status dispatch_mixed(int group, const CUtensorMap& mq, const CUtensorMap& mk
                          cudaStream_t stream) {
   if (group <= 8) return run_mixed<T, BS, 1>(mq, mk, mv, pp, dp, plan, stream);
   return run_mixed<T, BS, 2>(mq, mk, mv, pp, dp, plan, stream);
+}
+
+// Self-test of the bounded waits (pa_selftest_wait_timeout): two roles of one
+// CTA wait on mbarriers that nothing ever arrives on.  Role 0 (warp 0) gives
+// up after `limit_ns`; role 1 (warp 1) has the kernels' normal limit but polls
+// the CTA's abort word, which role 0 sets, so it gives up right after.  Each
+// role writes how long it waited.  No memory but the two words is touched.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, uint64_t* waited_ns) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_word;
+  volatile int* abort = &abort_word;
+  if (threadIdx.x == 0) {
+    pa::mbar_init(&bars[0], 1);
+    pa::mbar_init(&bars[1], 1);
+    *abort = 0;
+    pa::fence_barrier_init();
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    const uint64_t t0 = pa::global_timer_ns();
+    pa::mbar_wait(&bars[warp], 0, abort, warp == 0 ? limit_ns : pa::kWaitLimitNs);
+    if (waited_ns != nullptr) waited_ns[warp] = pa::global_timer_ns() - t0;
+  }
 }
 
 }  // namespace
@@ -911,6 +936,14 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
   }
   if (block_size == 16) return dispatch_mixed<__half, 16>(group, mq, mk, mv, pp, dp, plan, st);
   return dispatch_mixed<__half, 32>(group, mq, mk, mv, pp, dp, plan, st);
+}
+
+pa_status pa_selftest_wait_timeout(uint64_t limit_ns, uint64_t* waited_ns, pa_stream_t stream) {
+  if (limit_ns < 1000ull || limit_ns > 100000000ull) return PA_ERR_INVALID_ARG;
+  if (waited_ns != nullptr && (reinterpret_cast<uintptr_t>(waited_ns) & 7u) != 0)
+    return PA_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 64, 0, (cudaStream_t)stream>>>(limit_ns, waited_ns);
+  return launch_status();
 }
 
 pa_status pa_get_device_error(unsigned int* error_word, pa_stream_t stream) {

@@ -81,7 +81,7 @@ struct PrefillShape {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQ * TILE;
   static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE;
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 3 * NQ;
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 3 * NQ + 1;  // + the MMA drain barrier
   static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBAR * 8 + 16;
   static constexpr int BLOCKS_PER_TILE = BN / BS;
   static constexpr uint32_t TMEM_COLS = 512;    // S0 | S1 | O0 | O1
@@ -180,6 +180,33 @@ __device__ __forceinline__ void prefill_combine_tail(const PrefillParams& p, int
   }
 }
 
+// P = 2^(S * scale - m) for the 16-column chunks [C0, C1) of a softmax
+// thread's S row (in sv), written as 16-bit pairs over the row's S columns in
+// tensor memory (P of chunk cc goes to columns 8 cc .. 8 cc + 7, which the
+// thread has already read), with the row sum of P accumulated in four packed
+// fp32 partial sums.
+template <typename T, int C0, int C1>
+__device__ __forceinline__ void prefill_p_chunks(const uint32_t (&sv)[128], uint64_t sc2,
+                                                 uint64_t negm2, uint32_t t_s,
+                                                 uint64_t (&rsum)[4]) {
+#pragma unroll
+  for (int cc = C0; cc < C1; ++cc) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int x = cc * 16 + 2 * e;
+      float a, b;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), sc2, negm2),
+                a, b);
+      a = ex2_approx(a);
+      b = ex2_approx(b);
+      rsum[e & 3] = f2_add(rsum[e & 3], f2_pack(a, b));
+      pk[e] = MmaOp<T>::pack(a, b);
+    }
+    tmem_st8(t_s + cc * 8, pk);
+  }
+}
+
 // The work of one CTA: chunk rows tile * 256 .. tile * 256 + 255 of query
 // head h of sequence s, over the whole causal key range (nparts == 1) or over
 // part `part` of it, split into nparts runs of 128-key tiles (tail unit
@@ -201,8 +228,10 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   uint64_t* s_full = bars + 1 + 2 * NS;           // NQ
   uint64_t* p_full = s_full + NQ;                 // NQ
   uint64_t* o_final = p_full + NQ;                // NQ
+  uint64_t* mma_drain = o_final + NQ;             // 1 (used only after an abort)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Sh::NBAR);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(last_flag + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = p.cu_q_lens[s];
@@ -247,9 +276,11 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     }
     for (int w = 0; w < NQ; ++w) {
       mbar_init(&s_full[w], 1);
-      mbar_init(&p_full[w], 128);
+      mbar_init(&p_full[w], 4);  // one arrival per softmax warp
       mbar_init(&o_final[w], 1);
     }
+    mbar_init(mma_drain, 1);
+    *abort = 0;
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -261,6 +292,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  int armed = 0;  // TMA warp: ring items (K_j = 2j, V_j = 2j + 1) armed so far
   if (warp >= 8) {
     // producer warpgroup: TMA warp, MMA warp, two idle warps
     setmaxnreg_dec<Sh::PRODUCER_REGS>();
@@ -281,8 +313,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
                   q0 + i0 + w * BM, q_full, pol_q);
     }
     const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq;
-    bool alive = true;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; j < ntiles && armed == 2 * j; ++j) {
       const int b0 = (j0 + j) * Sh::BLOCKS_PER_TILE;
       const int nb = min(Sh::BLOCKS_PER_TILE, nblk_seq - b0);
       int phys = 0;
@@ -300,16 +331,18 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int item = 2 * j + kv, st = item % NS;
+        int ok = 1;
         if (lane == 0) {
-          if (item >= NS && alive) alive = mbar_wait(&ring_empty[st], ((item / NS) - 1) & 1);
-          mbar_arrive_expect_tx(&ring_full[st], bytes);
+          if (item >= NS) ok = mbar_wait(&ring_empty[st], ((item / NS) - 1) & 1, abort);
+          if (ok) mbar_arrive_expect_tx(&ring_full[st], bytes);
         }
-        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // gave up: load nothing more
         if (lane < 2 * nb) {
           tma_load_2d(smem + Sh::RING_OFF + st * Sh::TILE + (lane & 1) * Sh::HALF +
                           (lane >> 1) * BS * 128,
                       kv == 0 ? tm_k : tm_v, (lane & 1) * 64, row, &ring_full[st], pol_kv);
         }
+        armed = item + 1;
       }
     }
   } else if (warp == Sh::MMA_WARP) {
@@ -319,33 +352,36 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
       constexpr uint32_t idesc_pv = umma_idesc_f16(128, 128, kBf16, false, true);
       const uint32_t sq = smem_u32(smem + Sh::Q_OFF);
       const uint32_t ring = smem_u32(smem + Sh::RING_OFF);
-      bool alive = mbar_wait(q_full, 0);
-      if (alive) alive = mbar_wait(&ring_full[0], 0);  // K_0
-      tc_fence_after();
-      prefill_issue_s<Sh::HALF>(tmem, sq, ring, idesc_qk);
-      umma_commit(&s_full[0]);
-      prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring, idesc_qk);
-      umma_commit(&s_full[1]);
-      umma_commit(&ring_empty[0]);
-      for (int j = 0; j < ntiles; ++j) {
+      bool alive = mbar_wait(q_full, 0, abort) && mbar_wait(&ring_full[0], 0, abort);  // Q, K_0
+      if (alive) {
+        tc_fence_after();
+        prefill_issue_s<Sh::HALF>(tmem, sq, ring, idesc_qk);
+        umma_commit(&s_full[0]);
+        prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring, idesc_qk);
+        umma_commit(&s_full[1]);
+        umma_commit(&ring_empty[0]);
+      }
+      for (int j = 0; alive && j < ntiles; ++j) {
         const int it_v = 2 * j + 1, st_v = it_v % NS;
         const int it_k = 2 * j + 2, st_k = it_k % NS;
         const bool more = j + 1 < ntiles;
+        // V_j and K_{j+1} first: they are normally in shared memory long
+        // before P0_j, so nothing but P stands between a softmax hand-off and
+        // the next products
+        if (!mbar_wait(&ring_full[st_v], (it_v / NS) & 1, abort)) break;
+        if (more && !mbar_wait(&ring_full[st_k], (it_k / NS) & 1, abort)) break;
         // tile 0: PV0_j, then S0_{j+1}
-        if (alive) alive = mbar_wait(&p_full[0], j & 1);
-        if (alive) alive = mbar_wait(&ring_full[st_v], (it_v / NS) & 1);
+        if (!mbar_wait(&p_full[0], j & 1, abort)) break;
         tc_fence_after();
         prefill_issue_pv<Sh::HALF>(tmem + 256, tmem, ring + st_v * Sh::TILE, idesc_pv, j == 0);
         if (more) {
-          if (alive) alive = mbar_wait(&ring_full[st_k], (it_k / NS) & 1);
-          tc_fence_after();
           prefill_issue_s<Sh::HALF>(tmem, sq, ring + st_k * Sh::TILE, idesc_qk);
           umma_commit(&s_full[0]);
         } else {
           umma_commit(&o_final[0]);
         }
         // tile 1: PV1_j, then S1_{j+1}
-        if (alive) alive = mbar_wait(&p_full[1], j & 1);
+        if (!mbar_wait(&p_full[1], j & 1, abort)) break;
         tc_fence_after();
         prefill_issue_pv<Sh::HALF>(tmem + 384, tmem + 128, ring + st_v * Sh::TILE, idesc_pv,
                                    j == 0);
@@ -374,7 +410,9 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     float m_run = -INFINITY, l_run = 0.f;          // running max in log2 units
     bool alive = true;
     for (int j = 0; j < ntiles; ++j) {
-      if (alive) alive = mbar_wait(&s_full[w], j & 1);
+      // after a wait gave up every lane runs on through its (garbage) tiles
+      // alike, so the .aligned tensor-memory accesses stay converged
+      if (alive) alive = mbar_wait(&s_full[w], j & 1, abort);
       tc_fence_after();
       const int kbase = (j0 + j) * BN;
       if (w == 0 && j == ntiles - 1 && L - kbase < BN) {
@@ -382,7 +420,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
         // S0_j complete implies every earlier use of V_j's stage landed, so
         // this parity names the current phase.
         const int it_v = 2 * j + 1, st_v = it_v % NS;
-        if (alive) alive = mbar_wait(&ring_full[st_v], (it_v / NS) & 1);
+        if (alive) alive = mbar_wait(&ring_full[st_v], (it_v / NS) & 1, abort);
         const int first = L - kbase;
         uint8_t* vs = smem + Sh::RING_OFF + st_v * Sh::TILE;
         for (int idx = r; idx < (BN - first) * 16; idx += 128) {
@@ -404,66 +442,58 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
           if (kbase + e > limit) sv[e] = __float_as_uint(-INFINITY);
       }
       // row max: four independent chains of three-input max
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int e = 0; e < BN; e += 8) {
-        mx0 = fmax3(mx0, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
-        mx1 = fmax3(mx1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
-        mx2 = fmax3(mx2, __uint_as_float(sv[e + 4]), __uint_as_float(sv[e + 5]));
-        mx3 = fmax3(mx3, __uint_as_float(sv[e + 6]), __uint_as_float(sv[e + 7]));
+        mx[0] = fmax3(mx[0], __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+        mx[1] = fmax3(mx[1], __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+        mx[2] = fmax3(mx[2], __uint_as_float(sv[e + 4]), __uint_as_float(sv[e + 5]));
+        mx[3] = fmax3(mx[3], __uint_as_float(sv[e + 6]), __uint_as_float(sv[e + 7]));
       }
-      const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc;  // scale > 0 commutes
-      if (m_tile > m_run + 8.0f) {
-        // raise the running max; rescale l and O (O exists after tile 0, and
-        // S_w(j) complete implies PV_w(j-1) complete)
-        const float alpha = exp2f(m_run - m_tile);
+      const float m_tile = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;  // scale > 0 commutes
+      // The running max is raised only when the tile max exceeds it by more
+      // than 8 (log2 units): P <= 2^8 stays in 16-bit range and O is rarely
+      // rescaled (the stale max cancels in O / l).
+      const bool raise = m_tile > m_run + 8.0f;
+      float alpha = 1.f;
+      if (raise) {
+        alpha = exp2f(m_run - m_tile);  // 0 while m_run is -inf
         l_run *= alpha;
-        if (j > 0) {
-          // 32 columns at a time: the S row stays live in registers meanwhile
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(t_o + cc * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(t_o + cc * 32, ov);
-          }
-        }
         m_run = m_tile;
       }
-      // P = 2^(S * scale - m): packed FMA, SFU exp2, packed row sums
-      // a row with no visible key yet (only in a later part of a split
-      // unit) keeps m_run = -inf: use 0 so that its masked scores give 0
-      const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const uint64_t sc2 = f2_pack(sc, sc), negm2 = f2_pack(-m_use, -m_use);
-      uint64_t rsum[4] = {0, 0, 0, 0};  // four packed partial sums
+      // rescale O (S_w(j) complete implies PV_w(j-1) complete), 32 columns at
+      // a time, the S row staying live in registers; warp-uniform (the
+      // tensor-memory accesses are .aligned): rows whose max is unchanged
+      // multiply by 1
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(t_o + cc * 32, ov);
+          tmem_wait_ld_into<0>(ov);
 #pragma unroll
-      for (int cc = 0; cc < BN / 16; ++cc) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int x = cc * 16 + 2 * e;
-          float a, b;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[x]), __uint_as_float(sv[x + 1])), sc2,
-                           negm2),
-                    a, b);
-          a = ex2_approx(a);
-          b = ex2_approx(b);
-          rsum[e & 3] = f2_add(rsum[e & 3], f2_pack(a, b));
-          pk[e] = MmaOp<T>::pack(a, b);
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(t_o + cc * 32, ov);
         }
-        tmem_st8(t_s + cc * 8, pk);
       }
+      // P = 2^(S * scale - m): packed FMA, SFU exp2, packed row sums.  A row
+      // with no visible key yet (only in a later part of a split unit) keeps
+      // m_run = -inf: use 0 so that its masked scores give 0.
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      uint64_t rsum[4] = {0, 0, 0, 0};  // four packed partial row sums of P
+      prefill_p_chunks<T, 0, BN / 16>(sv, f2_pack(sc, sc), f2_pack(-m_use, -m_use), t_s, rsum);
       float l0, l1;
       f2_unpack(f2_add(f2_add(rsum[0], rsum[1]), f2_add(rsum[2], rsum[3])), l0, l1);
       l_run += l0 + l1;
+      // hand P to the MMA thread: every lane's stores are complete and ordered
+      // before the warp's one arrival
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[w]);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&p_full[w]);
     }
     // epilogue: O / l for the valid rows (one-shot barrier per Q tile)
-    if (alive) alive = mbar_wait(&o_final[w], 0);
+    if (alive) alive = mbar_wait(&o_final[w], 0, abort);
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(q0 + row) * p.num_q_heads + h) * D;
@@ -501,6 +531,19 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   }
   tc_fence_before();
   __syncthreads();
+  if (*abort) {
+    // a wait gave up: let this CTA's own loads and tensor-core products land
+    // before its shared and tensor memory are released
+    if (warp == Sh::TMA_WARP && lane == 0) {
+      mbar_drain(q_full, 0);
+      drain_ring<NS>(ring_full, armed);
+    }
+    if (warp == Sh::MMA_WARP && lane == 0) {
+      umma_commit(mma_drain);
+      mbar_drain(mma_drain, 0);
+    }
+    __syncthreads();
+  }
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, Sh::TMEM_COLS);

@@ -62,19 +62,53 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.  Returns
-// false (and records PA_DEVERR_WAIT_TIMEOUT) if it does not complete within
-// kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity to complete.
+//
+// `abort` is a shared-memory word of the waiting CTA (or of one decode worker
+// inside a CTA), zeroed before the CTA's first wait.  A wait that runs out of
+// time (`limit_ns` of the global timer) records PA_DEVERR_WAIT_TIMEOUT, sets
+// the word and returns false; every other wait of the same CTA polls the word
+// while it spins and returns false as soon as it is set.  So one lost arrival
+// costs the CTA one time limit, not one per role that waits behind it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) break;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) break;
   }
+  *abort = 1;
   record_error(PA_DEVERR_WAIT_TIMEOUT);
   return false;
+}
+
+// After an abort: wait (bounded, ignoring the abort word) for an operation of
+// this thread that is still in flight — a TMA load or a tensor-core product
+// that completes on `bar` by itself — so that the CTA does not release its
+// shared or tensor memory under it.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_error(PA_DEVERR_WAIT_TIMEOUT);
+      return;
+    }
+}
+
+// After an abort, by the thread that armed a TMA ring: wait (bounded) for
+// the last fill of every stage armed so far (ring positions < `armed`;
+// position i is the (i / NS)-th fill of stage i % NS), so that no load is
+// still landing in shared memory when the CTA or worker ends.
+template <int NS>
+__device__ __forceinline__ void drain_ring(uint64_t* full_bar, int armed) {
+  for (int st = 0; st < NS && st < armed; ++st) {
+    const int last = st + ((armed - 1 - st) / NS) * NS;  // last position on stage st
+    mbar_drain(&full_bar[st], (last / NS) & 1);
+  }
 }
 
 // Order this thread's generic-proxy shared-memory writes before later
@@ -300,6 +334,25 @@ __device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, uint32_t (&r)[N]) {
         "=r"(r[OFF + 24]), "=r"(r[OFF + 25]), "=r"(r[OFF + 26]), "=r"(r[OFF + 27]),
         "=r"(r[OFF + 28]), "=r"(r[OFF + 29]), "=r"(r[OFF + 30]), "=r"(r[OFF + 31])
       : "r"(taddr));
+}
+// Wait for this thread's tensor-memory loads and make r[OFF .. OFF + 31]
+// depend on the wait, so that no use of the loaded registers can be scheduled
+// before the data has arrived.
+template <int OFF, int N>
+__device__ __forceinline__ void tmem_wait_ld_into(uint32_t (&r)[N]) {
+  static_assert(OFF + 32 <= N, "range");
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[OFF + 0]), "+r"(r[OFF + 1]), "+r"(r[OFF + 2]), "+r"(r[OFF + 3]),
+        "+r"(r[OFF + 4]), "+r"(r[OFF + 5]), "+r"(r[OFF + 6]), "+r"(r[OFF + 7]),
+        "+r"(r[OFF + 8]), "+r"(r[OFF + 9]), "+r"(r[OFF + 10]), "+r"(r[OFF + 11]),
+        "+r"(r[OFF + 12]), "+r"(r[OFF + 13]), "+r"(r[OFF + 14]), "+r"(r[OFF + 15]),
+        "+r"(r[OFF + 16]), "+r"(r[OFF + 17]), "+r"(r[OFF + 18]), "+r"(r[OFF + 19]),
+        "+r"(r[OFF + 20]), "+r"(r[OFF + 21]), "+r"(r[OFF + 22]), "+r"(r[OFF + 23]),
+        "+r"(r[OFF + 24]), "+r"(r[OFF + 25]), "+r"(r[OFF + 26]), "+r"(r[OFF + 27]),
+        "+r"(r[OFF + 28]), "+r"(r[OFF + 29]), "+r"(r[OFF + 30]), "+r"(r[OFF + 31])
+      :
+      : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(

@@ -195,3 +195,11 @@ def test_binding_refuses_cpu_tensors(lib):
     kc = torch.zeros(4, 2, 16, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         pa.pa_copy_blocks(kc, kc.clone(), torch.zeros(1, 2, dtype=torch.int64))
+
+
+def test_wait_timeout_selftest_rejects_bad_limits(lib):
+    # limits outside 1 us .. 100 ms and a misaligned output are refused before any launch
+    for limit in (0, 999, 100_000_001, 2**63):
+        assert lib.pa_selftest_wait_timeout(limit, None, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_selftest_wait_timeout(1_000_000, ctypes.c_void_p(12), None) == \
+        pa.PA_ERR_INVALID_ARG

@@ -24,6 +24,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 _P, _I = ctypes.c_void_p, ctypes.c_int
 _C_TYPES = {
     "int": _I, "float": ctypes.c_float, "size_t": ctypes.c_size_t, "int64_t": ctypes.c_int64,
+    "uint64_t": ctypes.c_uint64,
     "pa_dtype": _I, "pa_stream_t": _P, "pa_status": _I, "void": None,
     "const char *": ctypes.c_char_p, "int *": ctypes.POINTER(_I),
     "size_t *": ctypes.POINTER(ctypes.c_size_t), "unsigned int *": ctypes.POINTER(ctypes.c_uint),
@@ -199,6 +200,10 @@ def test_every_wrapper_passes_the_c_arity_and_shape_sizes(rec):
 
     assert pa.pa_get_device_error() == 0
     _arity(rec, "pa_get_device_error")
+
+    pa.pa_selftest_wait_timeout(1_000_000)
+    a = _arity(rec, "pa_selftest_wait_timeout")
+    assert a[0] == 1_000_000 and a[1] is None
 
     host_only = {"pa_status_string", "pa_version", "pa_decode_partition_tokens"}
     called = {n for n, _ in rec.calls}
