@@ -339,6 +339,108 @@ def mixed_measure(dev, steps, warmup):
             "prefill_causal_flop": flops}
 
 
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the vendor figure the decode target is stated against
+
+
+def _decode_leg(name, w, lens_list, dev, steps, hbm_peak, *, tables=None, caches=None,
+                flush=None):
+    """pa_decode over one workload's batch (automatic partitions).  Returns ms,
+    GB/s of algorithmic K/V bytes (valid tokens only), fractions of the
+    measured and nominal HBM bandwidth and decode tokens/s (one layer).  With
+    `flush` (a device buffer larger than L2) every timed launch starts from a
+    cold L2 and is timed alone with events on the launching stream."""
+    import paged_kv_cache_397_b200 as pa
+    kc, vc = (w.key_cache.to(dev), w.value_cache.to(dev)) if caches is None else caches
+    bt = (w.block_tables if tables is None else tables).to(dev)
+    lens = torch.tensor(lens_list, dtype=torch.int32, device=dev)
+    q = w.query.to(dev)
+    out = torch.empty_like(q)
+    max_len = max(lens_list)
+    need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                       w.block_size, max_len)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    fn = lambda: pa.pa_decode(out, q, kc, vc, bt, lens, max_len, w.scale, workspace=ws)
+    stream = torch.cuda.current_stream()
+    for _ in range(5):
+        fn()
+    torch.cuda.synchronize()
+    if flush is None:
+        ms = time_steps(fn, steps, stream) / steps
+    else:
+        times = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+    esize = w.key_cache.element_size()
+    kv = 2 * w.num_kv_heads * w.head_dim * esize * sum(lens_list)
+    parts = math.ceil(max_len / pa.pa_decode_partition_tokens(w.num_seqs, w.num_kv_heads,
+                                                              w.block_size, max_len))
+    return {"workload": name, "ms": ms, "GBps": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / hbm_peak,
+            "hbm_frac_nominal": kv / ms / 1e6 / NOMINAL_HBM_GBS,
+            "decode_tokens_per_s": w.num_seqs / ms * 1e3, "kv_bytes": kv,
+            "partitions_per_longest_seq": parts, "l2": "cold (flushed)" if flush is not None
+            else "inputs larger than L2"}
+
+
+def decode_configs_measure(dev, steps, hbm_peak):
+    """Decode throughput on the other decode workloads: the Llama-2-13B shape
+    (fp16, 40 q = 40 kv heads, so one query head per KV head), the
+    shared-prefix batch after its copy-on-write (logical and unique bytes,
+    L2 cold and hot), and the 16 x 32768-token long-context batch (split-KV)
+    at block sizes 16 and 32."""
+    res = {}
+    w = synth.llama2_13b_decode()
+    res["llama2_13b_decode"] = _decode_leg(w.name, w, w.context_lens.tolist(), dev, steps,
+                                           hbm_peak)
+    del w
+    torch.cuda.empty_cache()
+    for B in (16, 32):
+        w = synth.long_context_decode(block_size=B)
+        res[f"long_context_decode_B{B}"] = _decode_leg(w.name, w, w.context_lens.tolist(), dev,
+                                                       steps, hbm_peak)
+        del w
+        torch.cuda.empty_cache()
+    # shared prefix: every sequence's last shared block is copied to a private
+    # block (pa_copy_blocks; timed on its own under copy_blocks) and remapped
+    import paged_kv_cache_397_b200 as pa
+    w = synth.shared_prefix_cow()
+    lens = w.context_lens.tolist()
+    kc, vc = w.key_cache.to(dev), w.value_cache.to(dev)
+    src = w.shared_blocks[w.cow_logical_block].repeat(w.num_seqs)
+    pa.pa_copy_blocks(kc, vc, torch.stack([src, w.cow_dst_blocks], 1).to(torch.int64).to(dev))
+    bt = w.block_tables.clone()
+    bt[:, w.cow_logical_block] = w.cow_dst_blocks.to(torch.int32)
+    # unique bytes: every physical block read once, valid tokens only
+    valid = {}
+    for s, L in enumerate(lens):
+        for j in range(-(-L // w.block_size)):
+            b = int(bt[s, j])
+            valid[b] = max(valid.get(b, 0), min(w.block_size, L - j * w.block_size))
+    unique = 2 * w.num_kv_heads * w.head_dim * 2 * sum(valid.values())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for mode, fl in (("cold", flush), ("hot", None)):
+        r = _decode_leg(w.name, w, lens, dev, steps, hbm_peak, tables=bt, caches=(kc, vc),
+                        flush=fl)
+        r["l2"] = "cold (256 MB written between launches)" if fl is not None else \
+            "hot (back-to-back launches; unique bytes fit the 126 MB L2 only in part)"
+        r["logical_kv_bytes"] = r.pop("kv_bytes")
+        r["logical_GBps"] = r.pop("GBps")
+        r["unique_kv_bytes"] = unique
+        r["unique_GBps"] = unique / r["ms"] / 1e6
+        r["hbm_frac"] = r["unique_GBps"] / hbm_peak
+        r["hbm_frac_nominal"] = r["unique_GBps"] / NOMINAL_HBM_GBS
+        res[f"shared_prefix_cow_decode_{mode}"] = r
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def copy_and_swap_measure(dev, steps):
     """Copy-on-write of the shared-prefix workload (128 block pairs) and swap
     of 256 blocks of the GQA decode shape out to pinned host memory and back."""
@@ -504,11 +606,18 @@ def main():
     stream = torch.cuda.current_stream()
     hbm_peak, bf16_peak, peak_kind = peaks()
 
+    # one step first: a device error (a bounded wait that gave up, a bad
+    # table entry) stops the run here instead of after the timed region
+    st.step()
+    err = pa.pa_get_device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x} after the first step")
+
     clocks = ClockSampler(local)
     clocks.start()
     # warm-up: at least W steps and at least --min-warmup-s under load
     t_end = time.time() + args.min_warmup_s
-    n = 0
+    n = 1
     while n < args.warmup or time.time() < t_end:
         st.step()
         n += 1
@@ -569,8 +678,12 @@ def main():
         torch.cuda.empty_cache()
         secondary = {"fp8_decode": fp8_decode_measure(dev, steps=50, warmup=5,
                                                       hbm_peak=hbm_peak)}
+        secondary["fp8_decode"]["hbm_frac_nominal"] = \
+            secondary["fp8_decode"]["value"] / NOMINAL_HBM_GBS
         torch.cuda.empty_cache()
         secondary["mixed_batch"] = mixed_measure(dev, steps=20, warmup=3)
+        torch.cuda.empty_cache()
+        secondary["decode_configs"] = decode_configs_measure(dev, steps=20, hbm_peak=hbm_peak)
         torch.cuda.empty_cache()
         secondary.update(copy_and_swap_measure(dev, steps=50))
 
@@ -588,11 +701,13 @@ def main():
                        "l2": "inputs larger than L2 (2.2 GB of K/V read per step, 126 MB L2)",
                        "parallelism": f"replicas x{world} (each rank its own batch)"},
             "hbm_frac": value / world / hbm_peak,
+            "hbm_frac_nominal": value / world / NOMINAL_HBM_GBS,
             "decode_tokens_per_s": world * w.num_seqs / (ms_step * 1e-3),
             "roofline": {"kernel": "pa_append_decode (decode_kernel with the fused append + "
                                    "decode_reduce_kernel)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
                          "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
+                         "frac_nominal": achieved / NOMINAL_HBM_GBS,
                          "peak_kind": f"hbm copy, {peak_kind}"},
             "prefill_chunk": prefill,
             "secondary": secondary,
