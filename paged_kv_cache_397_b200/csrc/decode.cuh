@@ -44,6 +44,7 @@
 
 #include <cuda_fp8.h>
 
+#include "cache_ops.cuh"
 #include "ptx.cuh"
 
 namespace pa {
@@ -61,13 +62,14 @@ struct DecodeParams {
   int max_parts;             // gridDim.x
   float scale_log2;          // softmax scale * log2(e) (FP8: also * k_scale)
   float v_scale;             // FP8: multiplies the output; 1 otherwise
+  float k_scale;             // FP8 with the fused append: the K cache's scale
   int len_add;               // tokens attended = seq_lens[s] + len_add (mixed batch: 1)
   // Fused append (pa_append_decode; null otherwise): the new token of
   // sequence s, at logical position seq_lens[s], is written into the cache
   // by the CTAs of its last partition before they read that block.
   const void* new_key;       // T[S][Hkv][D]
   const void* new_value;     // T[S][Hkv][D]
-  void* key_cache;           // T[num_blocks][Hkv][BS][D]
+  void* key_cache;           // T[num_blocks][Hkv][BS][D] (FP8: E4M3 codes)
   void* value_cache;
   int64_t* slot_out;         // [S] slot written (-1: none), or null
 };
@@ -377,6 +379,11 @@ struct DecodeShape {
   static constexpr int SMEM_BYTES = 1024 + BODY_BYTES + 2 * NS * 8 + 16;  // + abort word
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
+  // Consumer warp w takes ring positions w, w + NW, ... and waits on a
+  // stage's full barrier by the parity of the fill it wants; with NS a
+  // multiple of NW every stage is always consumed by the same warp, so no
+  // warp can wait on a stage two fills ahead (where that parity test would
+  // pass on an older phase).
   static_assert(NS % NW == 0, "ring depth vs consumer warps");
   static_assert(TT % BS == 0 && 32 % SB == 0 && ROWS % 16 == 0, "stage vs cache block");
   static_assert(HP == 1 || SB == 1, "a stage packs heads or blocks, not both");
@@ -647,30 +654,41 @@ __device__ __forceinline__ void reset_state(float (&o)[Tiles::D / 16][NT][4],
 }
 
 // Fused append, by the producer warp of the item that holds logical position
-// `pos` (the sequence's new token): write the token's K and V rows of KV
-// head kvh into its slot (block_tables[s][pos / BS], offset pos % BS), bit
-// copies, 16 bytes per lane, then order those writes before this CTA's TMA
-// reads of the block.  An out-of-pool block id is flagged and not written.
+// `pos` (the sequence's new token): write the token's K and V rows of the
+// item's KV heads (Tiles::HP of them, from pack index kvp) into its slot
+// (block_tables[s][pos / BS], offset pos % BS), 16 bytes per lane — bit
+// copies for fp16 / bf16 caches, E4M3 codes of value / scale (the rule of
+// pa_reshape_and_cache_fp8) for FP8 caches — then order those writes before
+// this CTA's TMA reads of the block.  An out-of-pool block id is flagged and
+// not written.
 template <class Tiles, int BS>
-__device__ __forceinline__ void append_new_token(const DecodeParams& p, int s, int kvh, int pos,
+__device__ __forceinline__ void append_new_token(const DecodeParams& p, int s, int kvp, int pos,
                                                  int lane) {
-  constexpr int CH = Tiles::D * 2 / 16;  // 16-byte chunks per K or V row
+  using T = typename Tiles::Elem;
+  constexpr int D = Tiles::D, HP = Tiles::HP;
+  constexpr int CB = Tiles::kHalfCache ? 2 : 1;  // cache bytes per element
+  constexpr int CH = D * CB / 16;                // 16-byte chunks per cache row
   const int32_t blk = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + pos / BS);
   const bool ok = blk >= 0 && blk < p.num_blocks;
   if (ok) {
-    const size_t row = ((size_t)blk * p.num_kv_heads + kvh) * BS + pos % BS;
-    const size_t src = (size_t)s * p.num_kv_heads + kvh;
-    for (int i = lane; i < 2 * CH; i += 32) {
-      const bool is_v = i >= CH;
-      const int c = is_v ? i - CH : i;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(is_v ? p.new_value : p.new_key) +
-                            src * CH + c);
+    for (int i = lane; i < 2 * HP * CH; i += 32) {
+      const bool is_v = i >= HP * CH;
+      const int r = is_v ? i - HP * CH : i;
+      const int h = kvp * HP + r / CH, c = r % CH;
+      const size_t row = ((size_t)blk * p.num_kv_heads + h) * BS + pos % BS;
+      const T* src = reinterpret_cast<const T*>(is_v ? p.new_value : p.new_key) +
+                     ((size_t)s * p.num_kv_heads + h) * D + c * (16 / CB);
+      uint4 v;
+      if constexpr (Tiles::kHalfCache)
+        v = __ldg(reinterpret_cast<const uint4*>(src));
+      else
+        v = quantize16_e4m3<T>(src, is_v ? p.v_scale : p.k_scale);
       reinterpret_cast<uint4*>(is_v ? p.value_cache : p.key_cache)[row * CH + c] = v;
     }
   } else if (lane == 0) {
     record_error(PA_DEVERR_BLOCK_RANGE);
   }
-  if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
+  if (lane == 0 && kvp == 0 && p.slot_out != nullptr)
     p.slot_out[s] = ok ? (int64_t)blk * BS + pos % BS : -1;
   fence_proxy_async_global();
   __syncwarp();
@@ -719,15 +737,13 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
       tma_prefetch_desc(tm_k);
       tma_prefetch_desc(tm_v);
     }
-    if constexpr (Tiles::kHalfCache) {
-      // fused append: the new token is the last position; skipped when the
-      // length was clamped (flagged by decode_len)
-      if (p.new_key != nullptr && part == nparts - 1) {
-        if (L >= 1 && p.seq_lens[s] + p.len_add == L)
-          append_new_token<Tiles, BS>(p, s, kvh, L - 1, lane);
-        else if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
-          p.slot_out[s] = -1;
-      }
+    // fused append: the new token is the last position; skipped when the
+    // length was clamped (flagged by decode_len)
+    if (p.new_key != nullptr && part == nparts - 1) {
+      if (L >= 1 && p.seq_lens[s] + p.len_add == L)
+        append_new_token<Tiles, BS>(p, s, kvh, L - 1, lane);
+      else if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
+        p.slot_out[s] = -1;
     }
     bool alive = true;
     const int armed = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s,
