@@ -256,15 +256,16 @@ def prefill_measure(dev, steps, warmup, block_size):
 
 
 def fp8_decode_measure(dev, steps, warmup, hbm_peak):
-    """The same GQA decode step over an FP8 (E4M3) pool: slot mapping, FP8
-    append, FP8 decode.  GB/s of FP8 K/V bytes read."""
+    """The same GQA decode step over an FP8 (E4M3) pool: the new token of
+    every sequence quantized and written, then the FP8 decode, in one launch
+    (pa_append_decode_fp8) plus the split-KV combine.  GB/s of FP8 K/V bytes
+    read."""
     import paged_kv_cache_397_b200 as pa
     w = synth.llama3_8b_gqa_decode_fp8()
     kc, vc, bt = w.key_cache.to(dev), w.value_cache.to(dev), w.block_tables.to(dev)
     ctx = w.context_lens.to(dev)
     lens = (w.context_lens + 1).to(dev)
     q, nk, nv = w.query.to(dev), w.new_key.to(dev), w.new_value.to(dev)
-    slots = torch.empty(w.num_seqs, dtype=torch.int64, device=dev)
     out = torch.empty_like(q)
     max_len = int(lens.max())
     need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
@@ -272,10 +273,8 @@ def fp8_decode_measure(dev, steps, warmup, hbm_peak):
     ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
 
     def step():
-        pa.pa_slot_mapping(slots, bt, ctx, w.block_size)
-        pa.pa_reshape_and_cache_fp8(nk, nv, kc, vc, slots, w.kv_scale, w.kv_scale)
-        pa.pa_decode_fp8(out, q, kc, vc, bt, lens, max_len, w.scale, w.kv_scale, w.kv_scale,
-                         workspace=ws)
+        pa.pa_append_decode_fp8(out, q, nk, nv, kc, vc, bt, ctx, max_len - 1, w.scale,
+                                w.kv_scale, w.kv_scale, workspace=ws)
 
     for _ in range(warmup):
         step()

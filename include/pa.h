@@ -299,6 +299,31 @@ pa_status pa_decode_fp8(void *out, const void *query, const uint8_t *key_cache,
                         pa_stream_t stream);
 
 /*
+ * pa_append_decode_fp8 — pa_append_decode over FP8 (E4M3) caches: one launch
+ * writes every sequence's new token as E4M3 codes (the encoding of
+ * pa_reshape_and_cache_fp8: value / scale, IEEE fp32 division, nearest code
+ * with ties to even, saturation at 448) and decodes over ctx_lens + 1 tokens.
+ *   "PagedAttention: KV cache as virtual memory", "Deep dive" (each decode
+ *   step appends one token) and "Interviewer follow-ups" (FP8 KV cache).
+ * new_key / new_value are T[num_seqs][num_kv_heads][head_dim] (T = dtype,
+ * fp16 or bf16, the query's type); key_cache / value_cache hold the codes.
+ * Output and cache contents are bit-identical to pa_slot_mapping +
+ * pa_reshape_and_cache_fp8 + pa_decode_fp8 with seq_lens = ctx_lens + 1,
+ * max_seq_len = max_ctx_len + 1 and the same partition_tokens and workspace
+ * (pa_decode_workspace_size with max_ctx_len + 1).  slot_mapping (int64[num_seqs],
+ * may be NULL) and the error behaviour are those of pa_append_decode.
+ * head_dim must be 128.
+ */
+pa_status pa_append_decode_fp8(void *out, const void *query, const void *new_key,
+                               const void *new_value, uint8_t *key_cache, uint8_t *value_cache,
+                               const int32_t *block_tables, const int32_t *ctx_lens,
+                               int64_t *slot_mapping, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               int max_blocks_per_seq, int max_ctx_len, int partition_tokens,
+                               float scale, float k_scale, float v_scale, pa_dtype dtype,
+                               void *workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * pa_decode_static_workspace — pa_decode for callers that cannot allocate
  * device memory.  (No counterpart on the pages: this is a library service,
  * not part of the paged-attention method.)

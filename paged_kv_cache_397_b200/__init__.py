@@ -30,7 +30,8 @@ __all__ = [
     "PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
     "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_append",
-    "pa_mixed_workspace_size", "pa_mixed_attention", "pa_append_decode", "BlockManager",
+    "pa_mixed_workspace_size", "pa_mixed_attention", "pa_append_decode", "pa_append_decode_fp8",
+    "BlockManager",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
 ]
@@ -67,6 +68,8 @@ _SIGS = {
                               _i, _f, _i, _p, _sz, _p]),
     "pa_append_decode": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                               _i, _i, _f, _i, _p, _sz, _p]),
+    "pa_append_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                                  _i, _i, _i, _f, _f, _f, _i, _p, _sz, _p]),
     "pa_mixed_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "pa_mixed_attention": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i,
                                 _i, _i, _i, _i, _f, _i, _p, _sz, _p]),
@@ -390,6 +393,41 @@ def pa_append_decode(out, query, new_key, new_value, key_cache, value_cache, blo
         _ptr(ctx_lens, "ctx_lens", torch.int32, 1), slot_ptr, S, hq, hkv, d, bs, nb,
         int(block_tables.shape[1]), int(max_ctx_len), int(partition_tokens), float(scale),
         _dtype_code(key_cache), ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def pa_append_decode_fp8(out, query, new_key, new_value, key_cache, value_cache, block_tables,
+                         ctx_lens, max_ctx_len, scale, k_scale, v_scale, slot_mapping=None,
+                         workspace=None, partition_tokens=0, stream=None):
+    """pa_append_decode over FP8 (E4M3, uint8) caches: the new tokens are
+    written as E4M3 codes of value / scale, then the decode runs over
+    ctx_lens + 1 tokens, in one launch (include/pa.h, pa_append_decode_fp8)."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if key_cache.dtype != torch.uint8:
+        raise ValueError("FP8 caches must be uint8 tensors of E4M3 codes")
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs][num_q_heads][head_dim]")
+    if out.dtype != query.dtype or new_key.dtype != query.dtype or new_value.dtype != query.dtype:
+        raise ValueError("out / new_key / new_value dtype must match the query")
+    S, hq = int(query.shape[0]), int(query.shape[1])
+    if new_key.shape != (S, hkv, d) or new_value.shape != (S, hkv, d):
+        raise ValueError("new_key/new_value must be [num_seqs][num_kv_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or ctx_lens.numel() != S:
+        raise ValueError("block_tables / ctx_lens do not match the batch")
+    need = pa_decode_workspace_size(S, hq, hkv, d, bs, int(max_ctx_len) + 1, partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    slot_ptr = _ptr(slot_mapping, "slot_mapping", torch.int64, 1) if slot_mapping is not None \
+        else None
+    _check("pa_append_decode_fp8", lib().pa_append_decode_fp8(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(new_key, "new_key"),
+        _ptr(new_value, "new_value"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(ctx_lens, "ctx_lens", torch.int32, 1), slot_ptr, S, hq, hkv, d, bs, nb,
+        int(block_tables.shape[1]), int(max_ctx_len), int(partition_tokens), float(scale),
+        float(k_scale), float(v_scale), _dtype_code(query), ws_ptr, ws_bytes, _stream(stream)))
     return out
 
 

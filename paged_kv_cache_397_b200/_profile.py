@@ -49,15 +49,18 @@ def decode_case(seqs: int, reps: int = 3):
 
 
 def decode_fp8_case(seqs: int, reps: int = 3):
+    """The bench's FP8 decode step (pa_append_decode_fp8) on a slice of its batch."""
     w = synth.llama3_8b_gqa_decode_fp8(num_seqs=seqs)
     d = torch.device("cuda:0")
     kc, vc, bt = w.key_cache.to(d), w.value_cache.to(d), w.block_tables.to(d)
-    lens = (w.context_lens + 1).to(d)
-    q = w.query.to(d)
+    ctx = w.context_lens.to(d)
+    lens = ctx + 1
+    q, nk, nv = w.query.to(d), w.new_key.to(d), w.new_value.to(d)
     out = torch.empty_like(q)
-    max_len = int(lens.max())
-    for _ in range(reps):
-        pa.pa_decode_fp8(out, q, kc, vc, bt, lens, max_len, w.scale, w.kv_scale, w.kv_scale)
+    max_ctx = int(w.context_lens.max())
+    for _ in range(reps):  # the same token rewritten into the same slot each time
+        pa.pa_append_decode_fp8(out, q, nk, nv, kc, vc, bt, ctx, max_ctx, w.scale, w.kv_scale,
+                                w.kv_scale)
     torch.cuda.synchronize()
     kv = 2 * w.num_kv_heads * w.head_dim * int(lens.sum())
     print(f"decode-fp8 case: {w.name}, K/V bytes per launch {kv}")

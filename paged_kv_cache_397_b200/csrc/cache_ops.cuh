@@ -155,6 +155,29 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
 // magnitudes above 448 saturating ("PagedAttention: KV cache as virtual
 // memory", "Interviewer follow-ups": an FP8 KV cache halves the bytes per
 // block; the encoding and the per-cache scale are this library's reading).
+// 16 consecutive fp16 / bf16 values at `in` (32-byte aligned) -> 16 E4M3
+// codes of value / scale: IEEE fp32 division, nearest code with ties to even,
+// saturation at +-448.
+template <typename T>
+__device__ __forceinline__ uint4 quantize16_e4m3(const T* in, float scale) {
+  uint4 raw[2];
+  raw[0] = __ldg(reinterpret_cast<const uint4*>(in));
+  raw[1] = __ldg(reinterpret_cast<const uint4*>(in) + 1);
+  const T* x = reinterpret_cast<const T*>(raw);
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(float(x[4 * q]) / scale, float(x[4 * q + 1]) / scale), __NV_SATFINITE,
+        __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(float(x[4 * q + 2]) / scale, float(x[4 * q + 3]) / scale), __NV_SATFINITE,
+        __NV_E4M3);
+    w[q] = (lo & 0xFFFF) | (hi << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 template <typename T>
 __global__ void reshape_and_cache_fp8_kernel(const T* __restrict__ key, const T* __restrict__ value,
                                              uint8_t* __restrict__ key_cache,
@@ -181,26 +204,9 @@ __global__ void reshape_and_cache_fp8_kernel(const T* __restrict__ key, const T*
   const int64_t src = th * head_dim + c * 16;
   const int64_t dst = ((b * num_kv_heads + h) * block_size + off) * head_dim + c * 16;
 #pragma unroll
-  for (int kv = 0; kv < 2; ++kv) {
-    const T* in = (kv == 0 ? key : value) + src;
-    const float sc = kv == 0 ? k_scale : v_scale;
-    uint4 raw[2];
-    raw[0] = __ldg(reinterpret_cast<const uint4*>(in));
-    raw[1] = __ldg(reinterpret_cast<const uint4*>(in) + 1);
-    const T* x = reinterpret_cast<const T*>(raw);
-    uint32_t w[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t lo = __nv_cvt_float2_to_fp8x2(
-          make_float2(float(x[4 * q]) / sc, float(x[4 * q + 1]) / sc), __NV_SATFINITE, __NV_E4M3);
-      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-          make_float2(float(x[4 * q + 2]) / sc, float(x[4 * q + 3]) / sc), __NV_SATFINITE,
-          __NV_E4M3);
-      w[q] = (lo & 0xFFFF) | (hi << 16);
-    }
+  for (int kv = 0; kv < 2; ++kv)
     *reinterpret_cast<uint4*>((kv == 0 ? key_cache : value_cache) + dst) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-  }
+        quantize16_e4m3<T>((kv == 0 ? key : value) + src, kv == 0 ? k_scale : v_scale);
 }
 
 // Copy-on-write block copies ("PagedAttention: Why Static Batching Wastes

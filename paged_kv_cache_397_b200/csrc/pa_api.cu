@@ -561,7 +561,7 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
     return PA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_INVALID_ARG;
-  if (app && (kv_fp8 || !app->new_key || !app->new_value || !aligned16(app->new_key) ||
+  if (app && (!app->new_key || !app->new_value || !aligned16(app->new_key) ||
               !aligned16(app->new_value)))
     return PA_ERR_INVALID_ARG;
   if ((long long)max_seq_len > (long long)max_blocks_per_seq * block_size)
@@ -615,6 +615,7 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
   p.max_parts = num_parts;
   p.scale_log2 = scale * (kv_fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   p.v_scale = kv_fp8 ? v_scale : 1.f;
+  p.k_scale = kv_fp8 ? k_scale : 1.f;
   p.len_add = app ? 1 : 0;  // fused append: seq_lens holds the context lengths
   p.new_key = app ? app->new_key : nullptr;
   p.new_value = app ? app->new_value : nullptr;
@@ -661,6 +662,22 @@ pa_status pa_append_decode(void* out, const void* query, const void* new_key,
                      num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                      max_blocks_per_seq, max_ctx_len + 1, partition_tokens, scale, 1.f, 1.f,
                      false, dtype, workspace, workspace_bytes, stream, &app);
+}
+
+pa_status pa_append_decode_fp8(void* out, const void* query, const void* new_key,
+                               const void* new_value, uint8_t* key_cache, uint8_t* value_cache,
+                               const int32_t* block_tables, const int32_t* ctx_lens,
+                               int64_t* slot_mapping, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               int max_blocks_per_seq, int max_ctx_len, int partition_tokens,
+                               float scale, float k_scale, float v_scale, pa_dtype dtype,
+                               void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+  if (max_ctx_len < 0 || max_ctx_len == INT_MAX) return PA_ERR_INVALID_ARG;  // decodes ctx + 1
+  const AppendArgs app{new_key, new_value, slot_mapping};
+  return decode_impl(out, query, key_cache, value_cache, block_tables, ctx_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                     max_blocks_per_seq, max_ctx_len + 1, partition_tokens, scale, k_scale,
+                     v_scale, true, dtype, workspace, workspace_bytes, stream, &app);
 }
 
 pa_status pa_decode_fp8(void* out, const void* query, const uint8_t* key_cache,

@@ -177,6 +177,29 @@ def test_append_decode_rejects_bad_arguments(lib):
     assert call(S=0) == pa.PA_OK
 
 
+def test_append_decode_fp8_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(out=FAKE, q=FAKE, nk=FAKE, nv=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE,
+                 sm=None, S=4, hq=8, hkv=2, d=128, bs=16, nb=64, mb=8, mc=100, pt=0,
+                 scale=0.1, ks=0.5, vs=0.25, dt=pa.PA_BF16, ws=None, wsb=0, st=None)
+        a.update(kw)
+        return lib.pa_append_decode_fp8(a["out"], a["q"], a["nk"], a["nv"], a["kc"], a["vc"],
+                                        a["bt"], a["cl"], a["sm"], a["S"], a["hq"], a["hkv"],
+                                        a["d"], a["bs"], a["nb"], a["mb"], a["mc"], a["pt"],
+                                        a["scale"], a["ks"], a["vs"], a["dt"], a["ws"],
+                                        a["wsb"], a["st"])
+
+    assert call(nk=None) == pa.PA_ERR_INVALID_ARG
+    assert call(nv=P(0x100008)) == pa.PA_ERR_INVALID_ARG          # misaligned
+    assert call(mc=8 * 16) == pa.PA_ERR_INVALID_ARG               # ctx + 1 does not fit
+    assert call(mc=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(ks=0.0) == pa.PA_ERR_INVALID_ARG                  # scales positive, finite
+    assert call(vs=float("inf")) == pa.PA_ERR_INVALID_ARG
+    assert call(dt=pa.PA_FP8_E4M3) == pa.PA_ERR_INVALID_ARG       # query type fp16 / bf16
+    assert call(d=64) == pa.PA_ERR_UNSUPPORTED                    # head_dim 128 only
+    assert call(S=0) == pa.PA_OK
+
+
 def test_cache_ops_reject_bad_arguments(lib):
     assert lib.pa_reshape_and_cache(None, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 16, 8, 1,
                                     None) == pa.PA_ERR_INVALID_ARG

@@ -180,6 +180,11 @@ def test_every_wrapper_passes_the_c_arity_and_shape_sizes(rec):
     a = _arity(rec, "pa_decode_fp8")
     assert a[6:18] == (S, hq, hkv, D, B, nb, width, 41, 0, 0.125, 0.5, 0.25)
 
+    pa.pa_append_decode_fp8(out, q, w.new_key, w.new_value, kc8, vc8, bt, ctx, 40, 0.125, 0.5,
+                            0.25, slot_mapping=slots)
+    a = _arity(rec, "pa_append_decode_fp8")
+    assert a[9:22] == (S, hq, hkv, D, B, nb, width, 40, 0, 0.125, 0.5, 0.25, pa.PA_BF16)
+
     p = synth.chunked_prefill(seed=1, block_size=16, hq=4, hkv=2, d=128, ctx_lens=[5, 0],
                               q_lens=[7, 3], dtype=torch.float16)
     pout = torch.empty_like(p.query)

@@ -155,3 +155,45 @@ def test_copy_blocks_on_fp8_caches():
     want_k[dst] = w.key_cache[src]
     want_v[dst] = w.value_cache[src]
     assert torch.equal(kc.cpu(), want_k) and torch.equal(vc.cpu(), want_v)
+
+
+# (dtype, block size, q heads, kv heads): packed kv-head pairs (16-token
+# blocks, G <= 4), unpacked 16-token blocks (G = 16), 32-token blocks
+FUSED_SHAPES = [(torch.bfloat16, 16, 32, 8), (torch.float16, 16, 16, 1), (torch.bfloat16, 32, 16, 4)]
+
+
+@pytest.mark.parametrize("dtype,B,hq,hkv", FUSED_SHAPES)
+@pytest.mark.parametrize("partition_tokens", [0, 64])
+def test_fused_append_decode_fp8_matches_three_calls(dtype, B, hq, hkv, partition_tokens):
+    # One launch (pa_append_decode_fp8) against slot mapping + FP8 scatter +
+    # FP8 decode: same cache bytes, same slots, same output bit for bit; and
+    # the output against the oracle's FP8 decode of the appended pool.
+    w = synth.random_decode(61 + B + hq, [0, 15, 16, 31, 100, 700], dtype=dtype, block_size=B,
+                            hq=hq, hkv=hkv, d=128, append=True, fp8_scale=1.0 / 16)
+    ctx = w.context_lens
+    lens = (ctx + 1).tolist()
+    q, nk, nv = to_dev(w.query), to_dev(w.new_key), to_dev(w.new_value)
+    bt, cd = to_dev(w.block_tables), to_dev(ctx)
+    mc = int(ctx.max())
+    # three calls
+    kc_a, vc_a = to_dev(w.key_cache), to_dev(w.value_cache)
+    slots_a = torch.empty(w.num_seqs, dtype=torch.int64, device=dev())
+    pa.pa_slot_mapping(slots_a, bt, cd, B)
+    pa.pa_reshape_and_cache_fp8(nk, nv, kc_a, vc_a, slots_a, w.kv_scale, w.kv_scale)
+    out_a = torch.empty_like(q)
+    pa.pa_decode_fp8(out_a, q, kc_a, vc_a, bt, to_dev(torch.tensor(lens, dtype=torch.int32)),
+                     mc + 1, w.scale, w.kv_scale, w.kv_scale, partition_tokens=partition_tokens)
+    # one launch
+    kc_b, vc_b = to_dev(w.key_cache), to_dev(w.value_cache)
+    slots_b = torch.full((w.num_seqs,), -7, dtype=torch.int64, device=dev())
+    out_b = torch.empty_like(q)
+    pa.pa_append_decode_fp8(out_b, q, nk, nv, kc_b, vc_b, bt, cd, mc, w.scale, w.kv_scale,
+                            w.kv_scale, slot_mapping=slots_b, partition_tokens=partition_tokens)
+    torch.cuda.synchronize()
+    assert torch.equal(slots_a, slots_b)
+    assert torch.equal(kc_a, kc_b) and torch.equal(vc_a, vc_b)
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+    # oracle: the appended pool decoded in fp64
+    w.key_cache, w.value_cache = kc_b.cpu(), vc_b.cpu()
+    ref = fp8_reference(w, lens, list(range(w.num_seqs)))
+    assert max_err(out_b.cpu(), ref) <= TOL[dtype]
