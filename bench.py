@@ -342,12 +342,14 @@ NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the vendor figure the decode target is s
 
 
 def _decode_leg(name, w, lens_list, dev, steps, hbm_peak, *, tables=None, caches=None,
-                flush=None):
+                flush=None, prefix=None):
     """pa_decode over one workload's batch (automatic partitions).  Returns ms,
     GB/s of algorithmic K/V bytes (valid tokens only), fractions of the
     measured and nominal HBM bandwidth and decode tokens/s (one layer).  With
     `flush` (a device buffer larger than L2) every timed launch starts from a
-    cold L2 and is timed alone with events on the launching stream."""
+    cold L2 and is timed alone with events on the launching stream.  With
+    `prefix` = (device int32 block ids, tokens) the batch runs through
+    pa_decode_shared_prefix instead."""
     import paged_kv_cache_397_b200 as pa
     kc, vc = (w.key_cache.to(dev), w.value_cache.to(dev)) if caches is None else caches
     bt = (w.block_tables if tables is None else tables).to(dev)
@@ -358,7 +360,11 @@ def _decode_leg(name, w, lens_list, dev, steps, hbm_peak, *, tables=None, caches
     need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
                                        w.block_size, max_len)
     ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    fn = lambda: pa.pa_decode(out, q, kc, vc, bt, lens, max_len, w.scale, workspace=ws)
+    if prefix is None:
+        fn = lambda: pa.pa_decode(out, q, kc, vc, bt, lens, max_len, w.scale, workspace=ws)
+    else:
+        fn = lambda: pa.pa_decode_shared_prefix(out, q, kc, vc, prefix[0], prefix[1], bt, lens,
+                                                max_len, w.scale, workspace=ws)
     stream = torch.cuda.current_stream()
     for _ in range(5):
         fn()
@@ -391,8 +397,9 @@ def decode_configs_measure(dev, steps, hbm_peak):
     """Decode throughput on the other decode workloads: the Llama-2-13B shape
     (fp16, 40 q = 40 kv heads, so one query head per KV head), the
     shared-prefix batch after its copy-on-write (logical and unique bytes,
-    L2 cold and hot), and the 16 x 32768-token long-context batch (split-KV)
-    at block sizes 16 and 32."""
+    L2 cold and hot, through pa_decode and through pa_decode_shared_prefix,
+    which reads each shared tile once per group of sequences), and the
+    16 x 32768-token long-context batch (split-KV) at block sizes 16 and 32."""
     res = {}
     w = synth.llama2_13b_decode()
     res["llama2_13b_decode"] = _decode_leg(w.name, w, w.context_lens.tolist(), dev, steps,
@@ -423,9 +430,15 @@ def decode_configs_measure(dev, steps, hbm_peak):
             valid[b] = max(valid.get(b, 0), min(w.block_size, L - j * w.block_size))
     unique = 2 * w.num_kv_heads * w.head_dim * 2 * sum(valid.values())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for mode, fl in (("cold", flush), ("hot", None)):
+    # the 49 blocks every sequence still shares after the copy-on-write
+    npre = w.cow_logical_block
+    pre = (w.shared_blocks[:npre].to(torch.int32).to(dev), npre * w.block_size)
+    for call, mode, fl, pf in (("", "cold", flush, None), ("", "hot", None, None),
+                               ("_shared_prefix_call", "cold", flush, pre),
+                               ("_shared_prefix_call", "hot", None, pre)):
         r = _decode_leg(w.name, w, lens, dev, steps, hbm_peak, tables=bt, caches=(kc, vc),
-                        flush=fl)
+                        flush=fl, prefix=pf)
+        r["call"] = "pa_decode_shared_prefix" if pf is not None else "pa_decode"
         r["l2"] = "cold (256 MB written between launches)" if fl is not None else \
             "hot (back-to-back launches; unique bytes fit the 126 MB L2 only in part)"
         r["logical_kv_bytes"] = r.pop("kv_bytes")
@@ -434,7 +447,7 @@ def decode_configs_measure(dev, steps, hbm_peak):
         r["unique_GBps"] = unique / r["ms"] / 1e6
         r["hbm_frac"] = r["unique_GBps"] / hbm_peak
         r["hbm_frac_nominal"] = r["unique_GBps"] / NOMINAL_HBM_GBS
-        res[f"shared_prefix_cow_decode_{mode}"] = r
+        res[f"shared_prefix_cow_decode{call}_{mode}"] = r
     del flush
     torch.cuda.empty_cache()
     return res

@@ -299,6 +299,41 @@ pa_status pa_decode_fp8(void *out, const void *query, const uint8_t *key_cache,
                         pa_stream_t stream);
 
 /*
+ * pa_decode_shared_prefix — pa_decode for a batch whose sequences all begin
+ * with the same cached prefix, stored once in shared physical blocks.
+ *   "PagedAttention: Why Static Batching Wastes Your KV Cache", "How does
+ *   copy-on-write eliminate duplicate prompt KV cache?" (sequences share the
+ *   blocks of a common prompt) and "vLLM PagedAttention Deep Dive",
+ *   "PagedAttention Mechanism".  Reading those blocks once for all sharers is
+ *   this library's design, not the pages'.
+ * Every sequence's first prefix_len tokens (a multiple of block_size, at most
+ * max_seq_len and at most each seq_lens[s]) are the K/V of the physical blocks
+ * prefix_blocks[0 .. prefix_len / block_size) — the same ids that lead every
+ * block_tables row; the rest of each sequence is read through block_tables as
+ * in pa_decode.  The split-KV partitions that lie wholly inside the prefix are
+ * computed once per group of sequences (up to 16 query columns per CTA: 16 /
+ * group sequences), each shared K/V tile read once for the group; the other
+ * partitions and the combine are pa_decode's.  With the same partition_tokens
+ * the output is bit-identical to pa_decode (each query column's arithmetic is
+ * unchanged).  When no partition lies inside the prefix, or group > 8, or the
+ * caches are not head_dim 128, this is pa_decode.
+ *   prefix_blocks  in  int32[prefix_len / block_size] (device memory)
+ * Every other argument, the workspace (pa_decode_workspace_size with the same
+ * sizes) and the error behaviour as pa_decode; a sequence shorter than a
+ * shared partition sets PA_DEVERR_SEQ_RANGE.  PA_ERR_INVALID_ARG for a
+ * negative prefix_len, one that is not a multiple of block_size or exceeds
+ * max_seq_len, or a null prefix_blocks with prefix_len > 0.
+ */
+pa_status pa_decode_shared_prefix(void *out, const void *query, const void *key_cache,
+                                  const void *value_cache, const int32_t *prefix_blocks,
+                                  int prefix_len, const int32_t *block_tables,
+                                  const int32_t *seq_lens, int num_seqs, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                  int max_blocks_per_seq, int max_seq_len, int partition_tokens,
+                                  float scale, pa_dtype dtype, void *workspace,
+                                  size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * pa_append_decode_fp8 — pa_append_decode over FP8 (E4M3) caches: one launch
  * writes every sequence's new token as E4M3 codes (the encoding of
  * pa_reshape_and_cache_fp8: value / scale, IEEE fp32 division, nearest code

@@ -31,6 +31,7 @@ __all__ = [
     "PA_ERR_OUT_OF_RANGE", "PA_ERR_CUDA", "PA_F16", "PA_BF16", "PA_FP8_E4M3",
     "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_append",
     "pa_mixed_workspace_size", "pa_mixed_attention", "pa_append_decode", "pa_append_decode_fp8",
+    "pa_decode_shared_prefix",
     "BlockManager",
     "PA_DEVERR_SLOT_RANGE", "PA_DEVERR_BLOCK_RANGE", "PA_DEVERR_SEQ_RANGE",
     "PA_DEVERR_WAIT_TIMEOUT",
@@ -70,6 +71,8 @@ _SIGS = {
                               _i, _i, _f, _i, _p, _sz, _p]),
     "pa_append_decode_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
                                   _i, _i, _i, _f, _f, _f, _i, _p, _sz, _p]),
+    "pa_decode_shared_prefix": (_i, [_p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i,
+                                     _i, _i, _i, _f, _i, _p, _sz, _p]),
     "pa_mixed_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "pa_mixed_attention": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i,
                                 _i, _i, _i, _i, _f, _i, _p, _sz, _p]),
@@ -392,6 +395,37 @@ def pa_append_decode(out, query, new_key, new_value, key_cache, value_cache, blo
         _ptr(value_cache, "value_cache"), _ptr(block_tables, "block_tables", torch.int32, 2),
         _ptr(ctx_lens, "ctx_lens", torch.int32, 1), slot_ptr, S, hq, hkv, d, bs, nb,
         int(block_tables.shape[1]), int(max_ctx_len), int(partition_tokens), float(scale),
+        _dtype_code(key_cache), ws_ptr, ws_bytes, _stream(stream)))
+    return out
+
+
+def pa_decode_shared_prefix(out, query, key_cache, value_cache, prefix_blocks, prefix_len,
+                            block_tables, seq_lens, max_seq_len, scale, workspace=None,
+                            partition_tokens=0, stream=None):
+    """pa_decode for a batch whose sequences share a leading prefix stored in
+    the physical blocks ``prefix_blocks`` (int32 CUDA tensor); the shared
+    partitions are computed once per group of sequences (include/pa.h)."""
+    nb, hkv, bs, d = _cache_dims(key_cache, value_cache)
+    if query.dim() != 3 or query.shape[2] != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs][num_q_heads][head_dim]")
+    if query.dtype != key_cache.dtype or out.dtype != key_cache.dtype:
+        raise ValueError("query/out dtype must match the cache")
+    S, hq = int(query.shape[0]), int(query.shape[1])
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.numel() != S:
+        raise ValueError("block_tables / seq_lens do not match the batch")
+    if prefix_blocks.numel() * bs < int(prefix_len):
+        raise ValueError("prefix_blocks holds fewer than prefix_len tokens")
+    need = pa_decode_workspace_size(S, hq, hkv, d, bs, int(max_seq_len), partition_tokens)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_shared_prefix", lib().pa_decode_shared_prefix(
+        _ptr(out, "out"), _ptr(query, "query"), _ptr(key_cache, "key_cache"),
+        _ptr(value_cache, "value_cache"), _ptr(prefix_blocks, "prefix_blocks", torch.int32, 1),
+        int(prefix_len), _ptr(block_tables, "block_tables", torch.int32, 2),
+        _ptr(seq_lens, "seq_lens", torch.int32, 1), S, hq, hkv, d, bs, nb,
+        int(block_tables.shape[1]), int(max_seq_len), int(partition_tokens), float(scale),
         _dtype_code(key_cache), ws_ptr, ws_bytes, _stream(stream)))
     return out
 

@@ -6,7 +6,7 @@
     python -m paged_kv_cache_397_b200._profile mixed --seqs 64
     python -m paged_kv_cache_397_b200._profile decode-llama2 --seqs 16
     python -m paged_kv_cache_397_b200._profile decode-long --seqs 2 [--block-size 16]
-    python -m paged_kv_cache_397_b200._profile decode-cow
+    python -m paged_kv_cache_397_b200._profile decode-cow [--shared-prefix]
 
 Each case builds a scaled-down copy of a bench workload (same shapes, head
 counts, length distribution and block shuffling; fewer sequences), runs the
@@ -131,8 +131,9 @@ def decode_long_case(seqs: int, block_size: int, reps: int = 3):
     print(f"decode-long case: {w.name}, K/V bytes per launch {kv}")
 
 
-def decode_cow_case(reps: int = 3):
-    """The shared-prefix batch (128 sequences) after its copy-on-write and remap."""
+def decode_cow_case(reps: int = 3, shared_prefix: bool = False):
+    """The shared-prefix batch (128 sequences) after its copy-on-write and
+    remap, through pa_decode or (shared_prefix) pa_decode_shared_prefix."""
     w = synth.shared_prefix_cow()
     d = torch.device("cuda:0")
     kc, vc = w.key_cache.to(d), w.value_cache.to(d)
@@ -140,7 +141,20 @@ def decode_cow_case(reps: int = 3):
     pa.pa_copy_blocks(kc, vc, torch.stack([src, w.cow_dst_blocks], 1).to(torch.int64).to(d))
     bt = w.block_tables.clone()
     bt[:, w.cow_logical_block] = w.cow_dst_blocks.to(torch.int32)
-    kv = _plain_decode(w, w.context_lens.tolist(), d, reps, tables=bt, caches=(kc, vc))
+    if shared_prefix:
+        lens = w.context_lens.tolist()
+        npre = w.cow_logical_block
+        ld = torch.tensor(lens, dtype=torch.int32, device=d)
+        q = w.query.to(d)
+        out = torch.empty_like(q)
+        pre = w.shared_blocks[:npre].to(torch.int32).to(d)
+        for _ in range(reps):
+            pa.pa_decode_shared_prefix(out, q, kc, vc, pre, npre * w.block_size, bt.to(d), ld,
+                                       max(lens), w.scale)
+        torch.cuda.synchronize()
+        kv = 2 * w.num_kv_heads * w.head_dim * 2 * sum(lens)
+    else:
+        kv = _plain_decode(w, w.context_lens.tolist(), d, reps, tables=bt, caches=(kc, vc))
     print(f"decode-cow case: {w.name}, logical K/V bytes per launch {kv}")
 
 
@@ -150,6 +164,7 @@ def main():
                                      "decode-long", "decode-cow"])
     ap.add_argument("--seqs", type=int, default=None)
     ap.add_argument("--block-size", type=int, default=16)
+    ap.add_argument("--shared-prefix", action="store_true")
     a = ap.parse_args()
     pa.lib()
     if a.case == "decode":
@@ -163,7 +178,7 @@ def main():
     elif a.case == "decode-long":
         decode_long_case(a.seqs or 2, a.block_size)
     elif a.case == "decode-cow":
-        decode_cow_case()
+        decode_cow_case(shared_prefix=a.shared_prefix)
     else:
         prefill_case(a.seqs or 4, a.block_size)
     if pa.pa_get_device_error():

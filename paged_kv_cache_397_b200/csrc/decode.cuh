@@ -72,6 +72,13 @@ struct DecodeParams {
   void* key_cache;           // T[num_blocks][Hkv][BS][D] (FP8: E4M3 codes)
   void* value_cache;
   int64_t* slot_out;         // [S] slot written (-1: none), or null
+  // Shared-prefix decode (pa_decode_shared_prefix): partition blockIdx.x of a
+  // launch is partition part_base + blockIdx.x of the sequence; the prefix
+  // launch reads the shared blocks from prefix_blocks and serves seq_group
+  // sequences per CTA.
+  int part_base = 0;
+  const int32_t* prefix_blocks = nullptr;
+  int seq_group = 1;
 };
 
 // ------------------------------------------------------------------ tiles
@@ -114,19 +121,26 @@ struct HalfTiles {
   __device__ static uint8_t* zero_chunk(uint8_t* v, int r, int idx) {
     return v + (idx >> 3) * BOX_BYTES + r * 128 + (idx & 7) * 16;
   }
-  // Q^T as the B operand: k = head dim in natural order
+  // Q^T as the B operand: k = head dim in natural order; query column g
+  // (g < G) is the row qbase + g * D
   template <int NT>
   __device__ static void load_q(uint32_t (&qf)[D / 16][NT][2], const T* qbase, int G,
                                 int lane) {
+    load_q_cols<NT>(qf, [&](int g) { return g < G ? qbase + (size_t)g * D : nullptr; }, lane);
+  }
+  // the same with column g taken from row_of(g) (nullptr: a zero column)
+  template <int NT, class RowOf>
+  __device__ static void load_q_cols(uint32_t (&qf)[D / 16][NT][2], RowOf row_of, int lane) {
     const int c4 = lane & 3, r4 = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int g = nt * 8 + r4;
+      const T* qrow = row_of(g);
 #pragma unroll
       for (int kt = 0; kt < D / 16; ++kt) {
         uint32_t b0 = 0, b1 = 0;
-        if (g < G) {
-          const uint32_t* row = reinterpret_cast<const uint32_t*>(qbase + (size_t)g * D);
+        if (qrow != nullptr) {
+          const uint32_t* row = reinterpret_cast<const uint32_t*>(qrow);
           b0 = __ldg(row + (kt * 16 + 2 * c4) / 2);
           b1 = __ldg(row + (kt * 16 + 2 * c4 + 8) / 2);
         }
@@ -407,7 +421,8 @@ __device__ __forceinline__ int decode_parts(int nblk_seq, int part_blocks) {
   return nblk_seq == 0 ? 1 : (nblk_seq + part_blocks - 1) / part_blocks;
 }
 
-// Producer side of one item: issue its nblk cache blocks, SB per ring stage
+// Producer side of one item: issue its nblk cache blocks (logical blocks
+// blk0 .. blk0 + nblk - 1 of the block-table row `table`), SB per ring stage
 // (the last stage of an item may hold fewer), into ring positions g0, g0 + 1,
 // ... (position i uses stage i % NS and is that stage's (i / NS)-th fill).
 // Block ids are fetched once, coalesced; entries past nblk are never read.
@@ -417,12 +432,13 @@ __device__ __forceinline__ int decode_parts(int nblk_seq, int part_blocks) {
 template <class Tiles, int BS, int NT>
 __device__ __forceinline__ int produce_item(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                             const DecodeParams& p, uint8_t* ring,
-                                            uint64_t* full_bar, uint64_t* empty_bar, int s,
-                                            int kvh, int blk0, int nblk, int g0, int lane,
-                                            uint64_t policy, bool& alive, volatile int* abort) {
+                                            uint64_t* full_bar, uint64_t* empty_bar,
+                                            const int32_t* table, int kvh, int blk0, int nblk,
+                                            int g0, int lane, uint64_t policy, bool& alive,
+                                            volatile int* abort) {
   using Shape = DecodeShape<Tiles, BS, NT>;
   constexpr int NS = Shape::NS, SB = Shape::SB;
-  const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+  const int32_t* bt = table + blk0;
   int armed = g0;
   for (int base = 0; base < nblk; base += 32) {
     int phys = 0;
@@ -563,14 +579,17 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
 
 // Merge the NW consumer warps' states of one item in shared memory `mg`
 // ([NW][8 NT][D + 2] floats) in warp order, then write the output row (one
-// partition) or the partition's (m, l, acc) to the workspace.  Opens with a
-// barrier of the consumer warps, so `mg` may alias the item's ring or the
-// previous item's merge area.
-template <class Tiles, int BS, int NT>
+// partition) or the partition's (m, l, acc) to the workspace.  Query column
+// g (g < cols) belongs to sequence s + g / G and query head kvh * G + g % G
+// (G = the item's query heads per sequence); single_of(seq) says whether that
+// sequence has one partition.  Opens with a barrier of the consumer warps, so
+// `mg` may alias the item's ring or the previous item's merge area.
+template <class Tiles, int BS, int NT, class SingleOf>
 __device__ __forceinline__ void merge_item(float* mg, float (&o)[Tiles::D / 16][NT][4],
                                            float (&m_run)[NT][2], float (&l_run)[NT][2],
                                            const DecodeParams& p, int s, int kvh, int part,
-                                           bool single, int ctid, uint32_t bar_consumers) {
+                                           int cols, SingleOf single_of, int ctid,
+                                           uint32_t bar_consumers) {
   using Shape = DecodeShape<Tiles, BS, NT>;
   using T = typename Tiles::Elem;
   constexpr int D = Shape::D, NW = Shape::NW;
@@ -610,7 +629,7 @@ __device__ __forceinline__ void merge_item(float* mg, float (&o)[Tiles::D / 16][
       }
   }
   named_barrier(bar_consumers, NW * 32);
-  for (int idx = ctid; idx < G * D; idx += NW * 32) {
+  for (int idx = ctid; idx < cols * D; idx += NW * 32) {
     const int g = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
@@ -624,12 +643,13 @@ __device__ __forceinline__ void merge_item(float* mg, float (&o)[Tiles::D / 16][
       den += sc * mg[(w * GP + g) * RS + D + 1];
     }
     num *= p.v_scale;
-    const int h = kvh * G + g;  // == (kvh * HP) * group + g
-    if (single) {
+    const int sq = s + g / G;
+    const int h = kvh * G + g % G;  // == (kvh * HP) * group + g for one sequence
+    if (single_of(sq)) {
       const float v = den > 0.f ? num / den : 0.f;
-      reinterpret_cast<T*>(p.out)[((size_t)s * p.num_q_heads + h) * D + d] = T(v);
+      reinterpret_cast<T*>(p.out)[((size_t)sq * p.num_q_heads + h) * D + d] = T(v);
     } else {
-      const size_t row = ((size_t)s * p.num_q_heads + h) * p.max_parts + part;
+      const size_t row = ((size_t)sq * p.num_q_heads + h) * p.max_parts + part;
       p.ws_acc[row * D + d] = num;
       if (d == 0) {
         p.ws_ml[row * 2] = M;
@@ -714,7 +734,7 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   volatile int* abort = reinterpret_cast<volatile int*>(empty_bar + NS);
   const int warp = tid >> 5, lane = tid & 31;
 
-  const int L = decode_len<BS>(p, s, tid == 0 && part == 0 && kvh == 0);
+  const int L = decode_len<BS>(p, s, tid == 0 && part == p.part_base && kvh == 0);
   const int nblk_seq = (L + BS - 1) / BS;
   const int nparts = decode_parts(nblk_seq, p.part_blocks);
   if (part >= nparts) return;
@@ -746,9 +766,10 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
         p.slot_out[s] = -1;
     }
     bool alive = true;
-    const int armed = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s,
-                                                  kvh, blk0, nblk, 0, lane,
-                                                  l2_policy_evict_first(), alive, abort);
+    const int armed = produce_item<Tiles, BS, NT>(
+        tm_k, tm_v, p, smem, full_bar, empty_bar,
+        p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, blk0, nblk, 0, lane,
+        l2_policy_evict_first(), alive, abort);
     named_barrier(bar_all, Shape::THREADS);  // the consumers are done
     if (*abort && lane == 0) drain_ring<NS>(full_bar, armed);
     return;
@@ -783,7 +804,7 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   // every consumer to finish reading it (after an abort a late load may still
   // land there; the output is garbage then, and the error word says so)
   merge_item<Tiles, BS, NT>(reinterpret_cast<float*>(smem), o, m_run, l_run, p, s, kvh, part,
-                            nparts == 1, tid, bar_consumers);
+                            G_item, [&](int) { return nparts == 1; }, tid, bar_consumers);
   named_barrier(bar_all, Shape::THREADS);  // lets the producer see the final abort word
 }
 
@@ -794,8 +815,105 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::mi
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  decode_item<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, blockIdx.x, blockIdx.y, blockIdx.z,
-                             threadIdx.x, 0, 1);
+  decode_item<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, p.part_base + blockIdx.x, blockIdx.y,
+                             blockIdx.z, threadIdx.x, 0, 1);
+}
+
+// Shared-prefix partitions (pa_decode_shared_prefix).  Every sequence of the
+// batch starts with the same physical blocks, prefix_blocks; partition `part`
+// (logical blocks part * part_blocks .. (part + 1) * part_blocks - 1, all of
+// them shared) is the same K/V for every sequence.  One CTA per (partition,
+// KV head, group of seq_group sequences) streams those tiles once and applies
+// them to the query heads of all the group's sequences, side by side in the
+// MMA's query columns (NT = 2: 16 columns).  Each column's arithmetic — the
+// score and P fragments, the per-warp online softmax, the merge over warps in
+// warp order — is exactly what pa_decode's CTA for that sequence does on the
+// same partition, so the partials (or, for a one-partition sequence, the
+// output row) are bit-identical to pa_decode's.
+template <class Tiles, int BS>
+__global__ void __launch_bounds__(DecodeShape<Tiles, BS, 2>::THREADS, Tiles::min_ctas(2))
+    prefix_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, DecodeParams p) {
+  constexpr int NT = 2;
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS;
+  static_assert(Shape::HP == 1, "fp16 / bf16 caches only");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Shape::BODY_BYTES);
+  uint64_t* empty_bar = full_bar + NS;
+  volatile int* abort = reinterpret_cast<volatile int*>(empty_bar + NS);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int part = blockIdx.x, kvh = blockIdx.y;
+  const int s0 = blockIdx.z * p.seq_group;
+  const int nseq = min(p.seq_group, p.num_seqs - s0);
+  const int G = p.group;
+  const int blk0 = part * p.part_blocks, nblk = p.part_blocks;
+  const int L_end = (blk0 + nblk) * BS;  // every token of the partition is valid
+
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    *abort = 0;
+    fence_barrier_init();
+    // every sequence must hold the whole shared partition
+    if (kvh == 0)
+      for (int j = 0; j < nseq; ++j)
+        if (decode_len<BS>(p, s0 + j, false) < L_end) record_error(PA_DEVERR_SEQ_RANGE);
+  }
+  named_barrier(0, Shape::THREADS);
+
+  if (warp == NW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    bool alive = true;
+    // the shared tiles are read by every group's CTA: keep them in L2
+    const int armed = produce_item<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, full_bar, empty_bar,
+                                                  p.prefix_blocks, kvh, blk0, nblk, 0, lane,
+                                                  l2_policy_evict_last(), alive, abort);
+    named_barrier(0, Shape::THREADS);  // the consumers are done
+    if (*abort && lane == 0) drain_ring<NS>(full_bar, armed);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  uint32_t qf[D / 16][NT][2];
+  const int cols = nseq * G;
+  Tiles::template load_q_cols<NT>(
+      qf,
+      [&](int g) -> const T* {
+        if (g >= cols) return nullptr;
+        return reinterpret_cast<const T*>(p.query) +
+               ((size_t)(s0 + g / G) * p.num_q_heads + (size_t)kvh * G + g % G) * D;
+      },
+      lane);
+  float m_run[NT][2], l_run[NT][2];
+  float o[D / 16][NT][4];
+  reset_state<Tiles, NT>(o, m_run, l_run);
+  const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
+  bool alive = true;
+  for (int i = warp; i < nstages; i += NW) {
+    const int st = i % NS;
+    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1, abort);
+    consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
+                                 (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane, G);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[st]);
+  }
+  merge_item<Tiles, BS, NT>(
+      reinterpret_cast<float*>(smem), o, m_run, l_run, p, s0, kvh, part, cols,
+      [&](int sq) {
+        return decode_parts((decode_len<BS>(p, sq, false) + BS - 1) / BS, p.part_blocks) == 1;
+      },
+      tid, 1);
+  named_barrier(0, Shape::THREADS);  // lets the producer see the final abort word
 }
 
 // Log-sum-exp combine of split-KV partitions, in partition order.  One warp

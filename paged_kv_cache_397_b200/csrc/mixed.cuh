@@ -127,9 +127,10 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
       }
       alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
       if (item < 0 || !alive) break;
-      const int next = produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, s,
-                                                   kvh, part * p.part_blocks, nblk, g, lane,
-                                                   policy, alive, abort);
+      const int next = produce_item<Tiles, BS, NT>(
+          tm_k, tm_v, p, smem, full_bar, empty_bar,
+          p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, part * p.part_blocks, nblk, g,
+          lane, policy, alive, abort);
       g = __shfl_sync(0xffffffffu, next, 0);  // lane 0's count (the lanes agree unless aborted)
     }
     named_barrier(bar_all, Shape::THREADS);  // the consumers are done
@@ -185,8 +186,8 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     g += nstages;
     // the opening barrier of merge_item also orders this item's read of
     // cur_item before thread 0 overwrites it for the next item
-    merge_item<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, nparts == 1, tid,
-                              bar_consumers);
+    merge_item<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, p.group,
+                              [&](int) { return nparts == 1; }, tid, bar_consumers);
   }
   named_barrier(bar_all, Shape::THREADS);  // lets the producer see the final abort word
 }

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <type_traits>
 #include <climits>
 #include <cmath>
 #include <mutex>
@@ -176,6 +177,49 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
   if (num_parts > 1) {
     const int units = p.num_seqs * p.num_q_heads;
     pa::decode_reduce_kernel<T, Shape::D>
+        <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
+            p, BS);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+// Shared-prefix decode: the prefix partitions [0, n_prefix) of every
+// sequence in prefix_decode_kernel (one CTA per partition, KV head and group
+// of p.seq_group sequences), the remaining partitions [n_prefix, num_parts)
+// in decode_kernel, then the combine.
+template <typename T, int BS>
+pa_status run_shared_prefix(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
+                            int num_parts, int n_prefix, cudaStream_t stream) {
+  using Tiles = pa::HalfTiles<T, 128, BS>;
+  using Shape = pa::DecodeShape<Tiles, BS, 2>;
+  auto kern = pa::prefix_decode_kernel<Tiles, BS>;
+  static std::atomic<unsigned long long> configured{0};
+  if (pa_status st = configure_kernel(configured, kern, Shape::SMEM_BYTES, 0); st != PA_OK)
+    return st;
+  const int groups = (p.num_seqs + p.seq_group - 1) / p.seq_group;
+  kern<<<dim3(n_prefix, p.num_kv_heads, groups), Shape::THREADS, Shape::SMEM_BYTES, stream>>>(
+      mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (num_parts > n_prefix) {
+    p.part_base = n_prefix;
+    auto launch = [&](auto nt_tag) -> pa_status {
+      constexpr int NT = decltype(nt_tag)::value;
+      using S = pa::DecodeShape<Tiles, BS, NT>;
+      auto dk = pa::decode_kernel<Tiles, BS, NT>;
+      static std::atomic<unsigned long long> conf{0};
+      if (pa_status st = configure_kernel(conf, dk, S::SMEM_BYTES, 0); st != PA_OK) return st;
+      dk<<<dim3(num_parts - n_prefix, p.num_kv_heads, p.num_seqs), S::THREADS, S::SMEM_BYTES,
+           stream>>>(mk, mv, p);
+      return launch_status();
+    };
+    const pa_status st = p.group <= 8 ? launch(std::integral_constant<int, 1>{})
+                                      : launch(std::integral_constant<int, 2>{});
+    if (st != PA_OK) return st;
+  }
+  if (num_parts > 1) {
+    const int units = p.num_seqs * p.num_q_heads;
+    pa::decode_reduce_kernel<T, 128>
         <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
             p, BS);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
@@ -540,6 +584,12 @@ struct AppendArgs {
   int64_t* slot_out;
 };
 
+// The shared prefix of pa_decode_shared_prefix (null for the other calls).
+struct PrefixArgs {
+  const int32_t* blocks;
+  int len;  // tokens, a multiple of block_size
+};
+
 pa_status decode_impl(void* out, const void* query, const void* key_cache,
                       const void* value_cache, const int32_t* block_tables,
                       const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
@@ -547,7 +597,7 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
                       int max_seq_len, int partition_tokens, float scale, float k_scale,
                       float v_scale, bool kv_fp8, pa_dtype dtype, void* workspace,
                       size_t workspace_bytes, pa_stream_t stream,
-                      const AppendArgs* app = nullptr) {
+                      const AppendArgs* app = nullptr, const PrefixArgs* prefix = nullptr) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
       max_blocks_per_seq <= 0 || max_seq_len < 0 || partition_tokens < 0 ||
       !valid_dtype(dtype) || !std::isfinite(scale))
@@ -565,6 +615,9 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
               !aligned16(app->new_value)))
     return PA_ERR_INVALID_ARG;
   if ((long long)max_seq_len > (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_INVALID_ARG;
+  if (prefix && (prefix->len < 0 || (prefix->len > 0 && prefix->blocks == nullptr) ||
+                 block_size <= 0 || prefix->len % block_size != 0 || prefix->len > max_seq_len))
     return PA_ERR_INVALID_ARG;
   if (num_seqs > 65535) return PA_ERR_INVALID_ARG;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
@@ -623,6 +676,23 @@ pa_status decode_impl(void* out, const void* query, const void* key_cache,
   p.value_cache = app ? const_cast<void*>(value_cache) : nullptr;
   p.slot_out = app ? app->slot_out : nullptr;
   auto st = (cudaStream_t)stream;
+  if (prefix && !kv_fp8 && head_dim == 128) {
+    // shared prefix: whole partitions inside it, batched across sequences
+    // when a CTA's 16 query columns hold at least two sequences
+    const int n_prefix = (prefix->len / block_size) / p.part_blocks;
+    p.seq_group = 16 / group;
+    if (n_prefix > 0 && p.seq_group >= 2) {
+      p.prefix_blocks = prefix->blocks;
+      if (dtype == PA_BF16) {
+        if (block_size == 16)
+          return run_shared_prefix<__nv_bfloat16, 16>(mk, mv, p, num_parts, n_prefix, st);
+        return run_shared_prefix<__nv_bfloat16, 32>(mk, mv, p, num_parts, n_prefix, st);
+      }
+      if (block_size == 16) return run_shared_prefix<__half, 16>(mk, mv, p, num_parts, n_prefix, st);
+      return run_shared_prefix<__half, 32>(mk, mv, p, num_parts, n_prefix, st);
+    }
+    p.seq_group = 1;  // otherwise: plain pa_decode
+  }
   if (kv_fp8) {
     if (dtype == PA_BF16) return dispatch_decode_fp8<__nv_bfloat16>(block_size, mk, mv, p, num_parts, st);
     return dispatch_decode_fp8<__half>(block_size, mk, mv, p, num_parts, st);
@@ -662,6 +732,21 @@ pa_status pa_append_decode(void* out, const void* query, const void* new_key,
                      num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                      max_blocks_per_seq, max_ctx_len + 1, partition_tokens, scale, 1.f, 1.f,
                      false, dtype, workspace, workspace_bytes, stream, &app);
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* query, const void* key_cache,
+                                  const void* value_cache, const int32_t* prefix_blocks,
+                                  int prefix_len, const int32_t* block_tables,
+                                  const int32_t* seq_lens, int num_seqs, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                  int max_blocks_per_seq, int max_seq_len, int partition_tokens,
+                                  float scale, pa_dtype dtype, void* workspace,
+                                  size_t workspace_bytes, pa_stream_t stream) {
+  const PrefixArgs prefix{prefix_blocks, prefix_len};
+  return decode_impl(out, query, key_cache, value_cache, block_tables, seq_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                     max_blocks_per_seq, max_seq_len, partition_tokens, scale, 1.f, 1.f, false,
+                     dtype, workspace, workspace_bytes, stream, nullptr, &prefix);
 }
 
 pa_status pa_append_decode_fp8(void* out, const void* query, const void* new_key,

@@ -177,6 +177,25 @@ def test_append_decode_rejects_bad_arguments(lib):
     assert call(S=0) == pa.PA_OK
 
 
+def test_decode_shared_prefix_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, pb=FAKE, pl=32, bt=FAKE, sl=FAKE, S=4,
+                 hq=8, hkv=2, d=128, bs=16, nb=64, mb=8, ml=100, pt=0, scale=0.1, dt=pa.PA_BF16,
+                 ws=None, wsb=0, st=None)
+        a.update(kw)
+        return lib.pa_decode_shared_prefix(a["out"], a["q"], a["kc"], a["vc"], a["pb"], a["pl"],
+                                           a["bt"], a["sl"], a["S"], a["hq"], a["hkv"], a["d"],
+                                           a["bs"], a["nb"], a["mb"], a["ml"], a["pt"],
+                                           a["scale"], a["dt"], a["ws"], a["wsb"], a["st"])
+
+    assert call(pl=-16) == pa.PA_ERR_INVALID_ARG
+    assert call(pl=24) == pa.PA_ERR_INVALID_ARG            # not a multiple of block_size
+    assert call(pl=112) == pa.PA_ERR_INVALID_ARG           # beyond max_seq_len
+    assert call(pb=None) == pa.PA_ERR_INVALID_ARG
+    assert call(ml=8 * 16 + 1) == pa.PA_ERR_INVALID_ARG    # as pa_decode
+    assert call(S=0) == pa.PA_OK
+
+
 def test_append_decode_fp8_rejects_bad_arguments(lib):
     def call(**kw):
         a = dict(out=FAKE, q=FAKE, nk=FAKE, nv=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE,

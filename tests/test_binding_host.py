@@ -166,6 +166,11 @@ def test_every_wrapper_passes_the_c_arity_and_shape_sizes(rec):
     a = _arity(rec, "pa_append_decode")
     assert a[9:18] == (S, hq, hkv, D, B, nb, width, 40, 0)
 
+    pa.pa_decode_shared_prefix(out, q, kc, vc, bt[0, :1].contiguous(), 16, bt, ctx + 1, 41,
+                               0.125, partition_tokens=16)
+    a = _arity(rec, "pa_decode_shared_prefix")
+    assert a[5] == 16 and a[8:18] == (S, hq, hkv, D, B, nb, width, 41, 16, 0.125)
+
     pa.pa_decode_static_workspace(out, q, kc, vc, bt, ctx + 1, 41, 0.125)
     a = _arity(rec, "pa_decode_static_workspace")
     assert a[6:15] == (S, hq, hkv, D, B, nb, width, 41, 0)
