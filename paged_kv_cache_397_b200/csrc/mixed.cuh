@@ -36,19 +36,118 @@ namespace pa {
 
 // Shared memory of one persistent decode worker: the TMA ring, a merge area
 // of its own (so the producer can stream the next item while the consumers
-// merge this one), ring and item-handoff mbarriers, the item slots, and the
-// item the consumers are working on.
+// merge this one; two warps' partial O at a time plus every warp's (m, l)),
+// ring and item-handoff mbarriers, the item slots, and the item the
+// consumers are working on.
 template <class Tiles, int BS, int NT>
 struct WorkerShape {
   using Dc = DecodeShape<Tiles, BS, NT>;
   static constexpr int QD = 2;  // item slots between producer and consumers
+  static constexpr int GP = NT * 8;
+  static constexpr int MERGE_BYTES = (2 * GP * (Dc::D + 2) + Dc::NW * GP * 2) * 4;
   static constexpr int MERGE_OFF = Dc::RING_BYTES;
-  static constexpr int BAR_OFF = MERGE_OFF + Dc::MERGE_BYTES;
+  static constexpr int BAR_OFF = MERGE_OFF + MERGE_BYTES;
   static constexpr int NBAR = 2 * Dc::NS + 2 * QD;
   static constexpr int ITEM_OFF = BAR_OFF + NBAR * 8;
   // item slots, the current item, the worker's abort word
   static constexpr int BYTES = (ITEM_OFF + (QD + 2) * 4 + 1023) / 1024 * 1024;
 };
+
+// Merge of one item's four consumer-warp states for a decode worker, through
+// a merge area half the size of merge_item's: every warp's (m, l) first, then
+// the partial O of warps 0-1 and, after them, of warps 2-3.  Each output
+// element is accumulated by the same thread in warp order w = 0, 1, 2, 3 with
+// the same operations as merge_item, so the result is bit-identical to
+// pa_decode's.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void merge_item_two_pass(float* mg, float (&o)[Tiles::D / 16][NT][4],
+                                                    float (&m_run)[NT][2], float (&l_run)[NT][2],
+                                                    const DecodeParams& p, int s, int kvh,
+                                                    int part, bool single, int ctid,
+                                                    uint32_t bar_consumers) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  using T = typename Tiles::Elem;
+  constexpr int D = Shape::D, NW = Shape::NW, GP = NT * 8, RS = D + 2;
+  constexpr int KMAX = GP * D / (NW * 32);  // output elements per thread (at most)
+  static_assert(NW == 4 && Shape::HP == 1, "four consumer warps, one KV head per item");
+  float* ml = mg + 2 * GP * RS;  // [NW][GP][2]
+  const int warp = ctid >> 5, lane = ctid & 31;
+  const int c4 = lane & 3, r4 = lane >> 2;
+  const int G = p.group;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float l = l_run[nt][j];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      l_run[nt][j] = l;
+    }
+  named_barrier(bar_consumers, NW * 32);  // every consumer is done with `mg`'s old contents
+  auto put_o = [&](int slot) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          mg[(slot * GP + nt * 8 + 2 * c4 + (e & 1)) * RS + Tiles::out_d(dt, e, r4)] =
+              o[dt][nt][e];
+  };
+  if (r4 == 0) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int g = nt * 8 + 2 * c4 + j;
+        ml[(warp * GP + g) * 2] = m_run[nt][j];
+        ml[(warp * GP + g) * 2 + 1] = l_run[nt][j];
+      }
+  }
+  if (warp < 2) put_o(warp);
+  named_barrier(bar_consumers, NW * 32);
+  float num[KMAX], den[KMAX];
+  auto accumulate = [&](int w0) {
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      const int idx = ctid + k * NW * 32;
+      if (idx >= G * D) continue;
+      const int g = idx / D, d = idx % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[(w * GP + g) * 2]);
+      const float m_use = M == -INFINITY ? 0.f : M;
+      if (w0 == 0) num[k] = den[k] = 0.f;
+#pragma unroll
+      for (int w = w0; w < w0 + 2; ++w) {
+        const float sc = exp2f(ml[(w * GP + g) * 2] - m_use);
+        num[k] += sc * mg[((w - w0) * GP + g) * RS + d];
+        den[k] += sc * ml[(w * GP + g) * 2 + 1];
+      }
+      if (w0 == 2) {
+        const float nv = num[k] * p.v_scale;
+        const int h = kvh * G + g;
+        if (single) {
+          const float v = den[k] > 0.f ? nv / den[k] : 0.f;
+          reinterpret_cast<T*>(p.out)[((size_t)s * p.num_q_heads + h) * D + d] = T(v);
+        } else {
+          const size_t row = ((size_t)s * p.num_q_heads + h) * p.max_parts + part;
+          p.ws_acc[row * D + d] = nv;
+          if (d == 0) {
+            p.ws_ml[row * 2] = M;
+            p.ws_ml[row * 2 + 1] = den[k];
+          }
+        }
+      }
+    }
+  };
+  accumulate(0);                          // warps 0 and 1
+  named_barrier(bar_consumers, NW * 32);  // their partial O has been read
+  if (warp >= 2) put_o(warp - 2);
+  named_barrier(bar_consumers, NW * 32);
+  accumulate(2);                          // warps 2 and 3, then the output
+}
 
 // A persistent decode worker (THREADS = 160 threads, `tid` 0..159): takes work
 // items i = atomicAdd(queue, 1) until i >= num_items; item i is partition
@@ -186,24 +285,34 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     g += nstages;
     // the opening barrier of merge_item also orders this item's read of
     // cur_item before thread 0 overwrites it for the next item
-    merge_item<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, p.group,
-                              [&](int) { return nparts == 1; }, tid, bar_consumers);
+    merge_item_two_pass<Tiles, BS, NT>(mg, o, m_run, l_run, p, s, kvh, part, nparts == 1, tid,
+                                       bar_consumers);
   }
   named_barrier(bar_all, Shape::THREADS);  // lets the producer see the final abort word
 }
 
+// CTA shape of the mixed launch.  With one query n-tile (groups up to 8) a
+// CTA of 16 warps hosts three decode workers, 12 consumer warps per SM as
+// three pa_decode CTAs have, and a prefill tile's softmax warpgroups get 200
+// registers by taking the other two warpgroups down to 56 (2 x 128 x 200 +
+// 256 x 56 = 512 x 128).  With two n-tiles the consumers need more registers:
+// 12 warps and two workers.
 template <typename T, int BS, int NT>
 struct MixedShape {
   using Pf = PrefillShape<T, BS>;
   using Tiles = HalfTiles<T, 128, BS>;
   using Dc = DecodeShape<Tiles, BS, NT>;
   using Wk = WorkerShape<Tiles, BS, NT>;
-  static constexpr int THREADS = Pf::THREADS;
+  static constexpr int THREADS = NT == 1 ? 512 : Pf::THREADS;
   static constexpr int WORKERS = THREADS / Dc::THREADS;  // decode workers per CTA
+  static constexpr uint32_t SOFT_REGS = Pf::SOFTMAX_REGS;
+  static constexpr uint32_t PROD_REGS = NT == 1 ? 56 : Pf::PRODUCER_REGS;
+  static constexpr int MIN_LAUNCH_REGS = NT == 1 ? 128 : Pf::MIN_LAUNCH_REGS;
+  static_assert(2 * 128 * SOFT_REGS + (THREADS - 256) * PROD_REGS <= THREADS * MIN_LAUNCH_REGS,
+                "register split exceeds the launch allocation");
   static constexpr int DEC_SMEM = 1024 + WORKERS * Wk::BYTES;
   static constexpr int SMEM_BYTES = Pf::SMEM_BYTES > DEC_SMEM ? Pf::SMEM_BYTES : DEC_SMEM;
-  static constexpr int MIN_LAUNCH_REGS = Pf::MIN_LAUNCH_REGS;
-  static_assert(WORKERS == 2, "two decode workers per CTA");
+  static_assert(WORKERS == (NT == 1 ? 3 : 2), "decode workers per CTA");
   static_assert(1 + 2 * WORKERS <= 16, "named barrier ids");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
@@ -233,11 +342,11 @@ __global__ void __launch_bounds__(MixedShape<T, BS, NT>::THREADS, 1)
     const int rest = b / plan.prefill_tiles;
     const int h = rest % pp.num_q_heads;
     const int s = plan.first_prefill_seq + rest / pp.num_q_heads;
-    prefill_tile<T, BS>(&tm_q, &tm_k, &tm_v, pp, smem, tile, h, s);
+    prefill_tile<T, BS, Sh::SOFT_REGS, Sh::PROD_REGS>(&tm_q, &tm_k, &tm_v, pp, smem, tile, h, s);
     return;
   }
   const int w = threadIdx.x / Sh::Dc::THREADS;
-  if (w >= Sh::WORKERS) return;  // the two spare warps
+  if (w >= Sh::WORKERS) return;  // the spare warps
   const int tid = threadIdx.x - w * Sh::Dc::THREADS;
   // decode rows: sequence s must own exactly query row s
   if (w == 0 && tid == 0) {

@@ -211,9 +211,12 @@ __device__ __forceinline__ void prefill_p_chunks(const uint32_t (&sv)[128], uint
 // head h of sequence s, over the whole causal key range (nparts == 1) or over
 // part `part` of it, split into nparts runs of 128-key tiles (tail unit
 // `slot`; the parts' partial rows are combined by the last one to finish).
-// Needs all THREADS threads of the CTA, 1024-byte aligned shared memory at
-// `smem` and all 512 tensor-memory columns.
-template <typename T, int BS>
+// Needs every thread of the CTA (12 warps, or more: warps past the producer
+// warpgroup idle), 1024-byte aligned shared memory at `smem` and all 512
+// tensor-memory columns.  SOFT_REGS / PROD_REGS: the setmaxnreg split between
+// the two softmax warpgroups and every other warpgroup of the CTA.
+template <typename T, int BS, uint32_t SOFT_REGS = PrefillShape<T, BS>::SOFTMAX_REGS,
+          uint32_t PROD_REGS = PrefillShape<T, BS>::PRODUCER_REGS>
 __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const PrefillParams& p,
                                              uint8_t* smem, int tile, int h, int s, int part = 0,
@@ -295,7 +298,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   int armed = 0;  // TMA warp: ring items (K_j = 2j, V_j = 2j + 1) armed so far
   if (warp >= 8) {
     // producer warpgroup: TMA warp, MMA warp, two idle warps
-    setmaxnreg_dec<Sh::PRODUCER_REGS>();
+    setmaxnreg_dec<PROD_REGS>();
   if (warp == Sh::TMA_WARP) {
     // ------------------------------------------------------------ TMA warp
     const uint64_t pol_kv = l2_policy_evict_last();
@@ -398,7 +401,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   }
   } else {
     // -------------------------------------------------- softmax warpgroups
-    setmaxnreg_inc<Sh::SOFTMAX_REGS>();
+    setmaxnreg_inc<SOFT_REGS>();
     const int w = warp >> 2;                       // Q tile of this warpgroup
     const int r = threadIdx.x & 127;               // row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
