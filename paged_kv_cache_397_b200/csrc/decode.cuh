@@ -815,8 +815,13 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, NT>::THREADS, Tiles::mi
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  // the split-KV combine that follows may be launched (it waits for this grid)
+  griddep_launch_dependents();
   decode_item<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, p.part_base + blockIdx.x, blockIdx.y,
                              blockIdx.z, threadIdx.x, 0, 1);
+  // launched to overlap a shared-prefix pass: finish only after it (so the
+  // combine, which waits for this grid, sees its partials)
+  griddep_wait();
 }
 
 // Shared-prefix partitions (pa_decode_shared_prefix).  Every sequence of the
@@ -866,6 +871,9 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, 2>::THREADS, Tiles::min
         if (decode_len<BS>(p, s0 + j, false) < L_end) record_error(PA_DEVERR_SEQ_RANGE);
   }
   named_barrier(0, Shape::THREADS);
+  // the rest of the sequences' partitions (decode_kernel) may start now: they
+  // write other partitions and wait for this grid before they finish
+  griddep_launch_dependents();
 
   if (warp == NW) {
     // ------------------------------------------------------------ producer
@@ -929,6 +937,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(REDUCE_WARPS * 32)
     decode_reduce_kernel(DecodeParams p, int block_size) {
   constexpr int VPL = D / 32;  // elements per lane: 4 (D = 128) or 2 (D = 64)
+  griddep_wait();  // launched early: the partials are complete only after this
   const int lane = threadIdx.x & 31;
   const int unit = blockIdx.x * REDUCE_WARPS + (threadIdx.x >> 5);
   if (unit >= p.num_seqs * p.num_q_heads) return;

@@ -162,6 +162,37 @@ int partition_tokens_for(int requested, int num_seqs, int num_kv_heads, int bloc
 // Partitions of a sequence of `len` tokens (at least one).
 long long num_partitions(int len, int pt) { return len == 0 ? 1 : ((long long)len + pt - 1) / pt; }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream still runs (from the moment all of that
+// kernel's CTAs have executed griddepcontrol.launch_dependents); it must
+// itself wait (griddepcontrol.wait) before it reads what that kernel writes.
+template <typename... KArgs, typename... Args>
+pa_status launch_overlapped(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? PA_OK
+                                                                                    : PA_ERR_CUDA;
+}
+
+// The split-KV combine after a decode launch, launched to overlap its tail
+// (decode_reduce_kernel waits for the decode grid before reading partials).
+template <typename T, int D>
+pa_status launch_combine(const pa::DecodeParams& p, int block_size, cudaStream_t stream) {
+  const int units = p.num_seqs * p.num_q_heads;
+  return launch_overlapped(pa::decode_reduce_kernel<T, D>,
+                           dim3((units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS),
+                           dim3(pa::REDUCE_WARPS * 32), 0, stream, p, block_size);
+}
+
 template <class Tiles, int BS, int NT>
 pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodeParams p,
                      int num_parts, cudaStream_t stream) {
@@ -174,13 +205,7 @@ pa_status run_decode(const CUtensorMap& mk, const CUtensorMap& mv, pa::DecodePar
   dim3 grid(num_parts, p.num_kv_heads / Tiles::HP, p.num_seqs);  // y: packs of HP kv heads
   kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (num_parts > 1) {
-    const int units = p.num_seqs * p.num_q_heads;
-    pa::decode_reduce_kernel<T, Shape::D>
-        <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
-            p, BS);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  }
+  if (num_parts > 1) return launch_combine<T, Shape::D>(p, BS, stream);
   return PA_OK;
 }
 
@@ -202,6 +227,8 @@ pa_status run_shared_prefix(const CUtensorMap& mk, const CUtensorMap& mv, pa::De
       mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (num_parts > n_prefix) {
+    // the other partitions overlap the prefix pass: they write other
+    // partials and wait for the prefix grid before their own grid ends
     p.part_base = n_prefix;
     auto launch = [&](auto nt_tag) -> pa_status {
       constexpr int NT = decltype(nt_tag)::value;
@@ -209,21 +236,14 @@ pa_status run_shared_prefix(const CUtensorMap& mk, const CUtensorMap& mv, pa::De
       auto dk = pa::decode_kernel<Tiles, BS, NT>;
       static std::atomic<unsigned long long> conf{0};
       if (pa_status st = configure_kernel(conf, dk, S::SMEM_BYTES, 0); st != PA_OK) return st;
-      dk<<<dim3(num_parts - n_prefix, p.num_kv_heads, p.num_seqs), S::THREADS, S::SMEM_BYTES,
-           stream>>>(mk, mv, p);
-      return launch_status();
+      return launch_overlapped(dk, dim3(num_parts - n_prefix, p.num_kv_heads, p.num_seqs),
+                               dim3(S::THREADS), S::SMEM_BYTES, stream, mk, mv, p);
     };
     const pa_status st = p.group <= 8 ? launch(std::integral_constant<int, 1>{})
                                       : launch(std::integral_constant<int, 2>{});
     if (st != PA_OK) return st;
   }
-  if (num_parts > 1) {
-    const int units = p.num_seqs * p.num_q_heads;
-    pa::decode_reduce_kernel<T, 128>
-        <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
-            p, BS);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  }
+  if (num_parts > 1) return launch_combine<T, 128>(p, BS, stream);
   return PA_OK;
 }
 
