@@ -81,7 +81,7 @@ struct PrefillShape {
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQ * TILE;
   static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE;
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 3 * NQ + 1;  // + the MMA drain barrier
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 4 * NQ + 1;  // + the MMA drain barrier
   static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBAR * 8 + 16;
   static constexpr int BLOCKS_PER_TILE = BN / BS;
   static constexpr uint32_t TMEM_COLS = 512;    // S0 | S1 | O0 | O1
@@ -100,14 +100,14 @@ __device__ __forceinline__ void prefill_issue_s(uint32_t d_tmem, uint32_t q_smem
   }
 }
 
-// O_w += P_w V: 8 K-steps of 16 keys; P from tensor memory (8 columns of
-// packed 16-bit pairs per step), V MN-major with its two 64-column halves
-// HALF bytes apart.
-template <int HALF>
+// O_w += P_w V over the K-steps [K0, K1) of 16 keys; P from tensor memory (8
+// columns of packed 16-bit pairs per step), V MN-major with its two 64-column
+// halves HALF bytes apart.
+template <int HALF, int K0, int K1>
 __device__ __forceinline__ void prefill_issue_pv(uint32_t o_tmem, uint32_t p_tmem,
                                                  uint32_t v_smem, uint32_t idesc, bool first) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
+  for (int kk = K0; kk < K1; ++kk)
     umma_ts(o_tmem, p_tmem + kk * 8, umma_desc_sw128(v_smem + kk * 16 * 128, HALF, 1024), idesc,
             (!first || kk > 0) ? 1u : 0u);
 }
@@ -231,7 +231,8 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   uint64_t* s_full = bars + 1 + 2 * NS;           // NQ
   uint64_t* p_full = s_full + NQ;                 // NQ
   uint64_t* o_final = p_full + NQ;                // NQ
-  uint64_t* mma_drain = o_final + NQ;             // 1 (used only after an abort)
+  uint64_t* p_half = o_final + NQ;                // NQ: P of the tile's first 64 keys
+  uint64_t* mma_drain = p_half + NQ;              // 1 (used only after an abort)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Sh::NBAR);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(last_flag + 1);
@@ -280,6 +281,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     for (int w = 0; w < NQ; ++w) {
       mbar_init(&s_full[w], 1);
       mbar_init(&p_full[w], 4);  // one arrival per softmax warp
+      mbar_init(&p_half[w], 4);
       mbar_init(&o_final[w], 1);
     }
     mbar_init(mma_drain, 1);
@@ -373,21 +375,31 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
         // the next products
         if (!mbar_wait(&ring_full[st_v], (it_v / NS) & 1, abort)) break;
         if (more && !mbar_wait(&ring_full[st_k], (it_k / NS) & 1, abort)) break;
-        // tile 0: PV0_j, then S0_{j+1}
+        // tile 0: PV0_j over the first 64 keys as soon as their P is
+        // written, the rest with P complete, then S0_{j+1}
+        if (!mbar_wait(&p_half[0], j & 1, abort)) break;
+        tc_fence_after();
+        prefill_issue_pv<Sh::HALF, 0, 4>(tmem + 256, tmem, ring + st_v * Sh::TILE, idesc_pv,
+                                         j == 0);
         if (!mbar_wait(&p_full[0], j & 1, abort)) break;
         tc_fence_after();
-        prefill_issue_pv<Sh::HALF>(tmem + 256, tmem, ring + st_v * Sh::TILE, idesc_pv, j == 0);
+        prefill_issue_pv<Sh::HALF, 4, 8>(tmem + 256, tmem, ring + st_v * Sh::TILE, idesc_pv,
+                                         false);
         if (more) {
           prefill_issue_s<Sh::HALF>(tmem, sq, ring + st_k * Sh::TILE, idesc_qk);
           umma_commit(&s_full[0]);
         } else {
           umma_commit(&o_final[0]);
         }
-        // tile 1: PV1_j, then S1_{j+1}
+        // tile 1: PV1_j in the same two parts, then S1_{j+1}
+        if (!mbar_wait(&p_half[1], j & 1, abort)) break;
+        tc_fence_after();
+        prefill_issue_pv<Sh::HALF, 0, 4>(tmem + 384, tmem + 128, ring + st_v * Sh::TILE,
+                                         idesc_pv, j == 0);
         if (!mbar_wait(&p_full[1], j & 1, abort)) break;
         tc_fence_after();
-        prefill_issue_pv<Sh::HALF>(tmem + 384, tmem + 128, ring + st_v * Sh::TILE, idesc_pv,
-                                   j == 0);
+        prefill_issue_pv<Sh::HALF, 4, 8>(tmem + 384, tmem + 128, ring + st_v * Sh::TILE,
+                                         idesc_pv, false);
         umma_commit(&ring_empty[st_v]);
         if (more) {
           prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring + st_k * Sh::TILE, idesc_qk);
@@ -484,7 +496,15 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
       // m_run = -inf: use 0 so that its masked scores give 0.
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       uint64_t rsum[4] = {0, 0, 0, 0};  // four packed partial row sums of P
-      prefill_p_chunks<T, 0, BN / 16>(sv, f2_pack(sc, sc), f2_pack(-m_use, -m_use), t_s, rsum);
+      const uint64_t sc2 = f2_pack(sc, sc), negm2 = f2_pack(-m_use, -m_use);
+      prefill_p_chunks<T, 0, BN / 32>(sv, sc2, negm2, t_s, rsum);
+      // the first 64 keys' P (columns 0-31) goes to the MMA thread while the
+      // rest is computed
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&p_half[w]);
+      prefill_p_chunks<T, BN / 32, BN / 16>(sv, sc2, negm2, t_s, rsum);
       float l0, l1;
       f2_unpack(f2_add(f2_add(rsum[0], rsum[1]), f2_add(rsum[2], rsum[3])), l0, l1);
       l_run += l0 + l1;
