@@ -20,7 +20,9 @@
 //    shared memory) and O_w += P_w V_j (P from tensor memory, V an MN-major
 //    shared-memory operand).  Issue order: S0_0, S1_0, then for every tile
 //    PV0_j, S0_{j+1}, PV1_j, S1_{j+1}: while one softmax warpgroup works on
-//    its scores, the tensor core runs the other tile's products.
+//    its scores, the tensor core runs the other tile's products.  PV_w(j)
+//    goes out in two parts: its first 4 K-steps (keys 0-63) once the softmax
+//    warps report that part of P stored, the rest with P complete.
 //    Completion is signalled with tcgen05.commit on mbarriers.
 //  * warps 0-3 and 4-7 (softmax, one warpgroup per Q tile): thread r owns
 //    query row r = TMEM lane r.  It loads its S row (tcgen05.ld), masks only
