@@ -419,7 +419,7 @@ pa_status pa_decode_static_workspace(void *out, const void *query, const void *k
  *              workspace's counters on `stream` first).  Calls sharing a
  *              workspace must be ordered.  Without one every unit runs
  *              whole; the two differ only in fp32 rounding order.
- * head_dim must be 128.
+ * head_dim 64 or 128 (else PA_ERR_UNSUPPORTED).
  */
 pa_status pa_prefill_workspace_size(int head_dim, size_t *bytes);
 pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,

@@ -318,11 +318,11 @@ void plan_prefill_split(pa::PrefillParams& p, long long units, bool have_ws) {
   p.n_full = (int)(best_k > 1 ? units - rem : units);
 }
 
-template <typename T, int BS>
+template <typename T, int BS, int D>
 pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       pa::PrefillParams p, cudaStream_t stream) {
-  using Sh = pa::PrefillShape<T, BS>;
-  auto kern = pa::prefill_kernel<T, BS>;
+  using Sh = pa::PrefillShape<T, BS, D>;
+  auto kern = pa::prefill_kernel<T, BS, D>;
   // the kernel's setmaxnreg split assumes at least MIN_LAUNCH_REGS registers per thread
   static std::atomic<unsigned long long> configured{0};  // per instantiation
   if (pa_status st = configure_kernel(configured, kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS);
@@ -336,6 +336,22 @@ pa_status run_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
     return PA_ERR_CUDA;
   kern<<<(unsigned)grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return launch_status();
+}
+
+template <typename T, int D>
+pa_status dispatch_prefill_bs(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const pa::PrefillParams& p, int block_size, cudaStream_t st) {
+  if (block_size == 16) return run_prefill<T, 16, D>(mq, mk, mv, p, st);
+  return run_prefill<T, 32, D>(mq, mk, mv, p, st);
+}
+pa_status dispatch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           const pa::PrefillParams& p, pa_dtype dtype, int block_size,
+                           int head_dim, cudaStream_t st) {
+  if (dtype == PA_BF16)
+    return head_dim == 64 ? dispatch_prefill_bs<__nv_bfloat16, 64>(mq, mk, mv, p, block_size, st)
+                          : dispatch_prefill_bs<__nv_bfloat16, 128>(mq, mk, mv, p, block_size, st);
+  return head_dim == 64 ? dispatch_prefill_bs<__half, 64>(mq, mk, mv, p, block_size, st)
+                        : dispatch_prefill_bs<__half, 128>(mq, mk, mv, p, block_size, st);
 }
 
 // Split-KV partition length of the decode rows of a mixed batch: as for
@@ -880,7 +896,7 @@ pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
   if ((long long)max_ctx_len >= (long long)max_blocks_per_seq * block_size)
     return PA_ERR_INVALID_ARG;
   if (num_seqs > 65535 || num_q_heads > 65535) return PA_ERR_INVALID_ARG;
-  if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
   if ((long long)num_blocks * num_kv_heads * block_size > INT_MAX) return PA_ERR_INVALID_ARG;
   if ((long long)total_q * num_q_heads * head_dim > INT_MAX) return PA_ERR_INVALID_ARG;
@@ -918,13 +934,7 @@ pa_status pa_prefill_chunk(void* out, const void* query, const void* key_cache,
     p.counters = nullptr;
     p.ws_o = p.ws_ml = nullptr;
   }
-  auto st = (cudaStream_t)stream;
-  if (dtype == PA_BF16) {
-    if (block_size == 16) return run_prefill<__nv_bfloat16, 16>(mq, mk, mv, p, st);
-    return run_prefill<__nv_bfloat16, 32>(mq, mk, mv, p, st);
-  }
-  if (block_size == 16) return run_prefill<__half, 16>(mq, mk, mv, p, st);
-  return run_prefill<__half, 32>(mq, mk, mv, p, st);
+  return dispatch_prefill(mq, mk, mv, p, dtype, block_size, head_dim, (cudaStream_t)stream);
 }
 
 pa_status pa_mixed_workspace_size(int num_decode_seqs, int num_q_heads, int num_kv_heads,

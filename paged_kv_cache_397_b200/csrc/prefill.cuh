@@ -61,9 +61,10 @@ struct PrefillParams {
   int* counters;      // [tail units] parts finished; zero at launch
 };
 
-template <typename T, int BS>
+template <typename T, int BS, int D_ = 128>
 struct PrefillShape {
-  static constexpr int D = 128;
+  static constexpr int D = D_;                  // head_dim: 64 or 128
+  static constexpr int NH = D / 64;             // 64-column (128-byte) halves of a row
   static constexpr int BM = 128;                // rows per Q tile
   static constexpr int NQ = 2;                  // Q tiles per CTA
   static constexpr int BN = 128;                // keys per K/V tile
@@ -78,24 +79,27 @@ struct PrefillShape {
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= THREADS * MIN_LAUNCH_REGS,
                 "register split exceeds the launch allocation");
   static constexpr int HALF = 128 * 128;        // 128 rows x 64 columns x 2 bytes
-  static constexpr int TILE = 2 * HALF;         // 128 x 128 x 2 bytes = 32 KB
-  static constexpr int NSTAGE = 4;              // K/V ring stages (K_j, V_j alternate)
+  static constexpr int TILE = NH * HALF;        // 128 rows x D columns x 2 bytes (16 or 32 KB)
+  // K/V ring stages (K_j, V_j alternate): the same 128 KB at either head_dim
+  static constexpr int NSTAGE = 4 * (2 / NH);
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = NQ * TILE;
   static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE;
   static constexpr int NBAR = 1 + 2 * NSTAGE + 4 * NQ + 1;  // + the MMA drain barrier
   static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBAR * 8 + 16;
   static constexpr int BLOCKS_PER_TILE = BN / BS;
-  static constexpr uint32_t TMEM_COLS = 512;    // S0 | S1 | O0 | O1
-  static_assert(2 * BLOCKS_PER_TILE <= 32, "one TMA box per lane");
+  static constexpr uint32_t TMEM_COLS = 512;    // S0 | S1 | O0 | O1 (O: D columns of 128)
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(NH * BLOCKS_PER_TILE <= 32, "one TMA box per lane");
 };
 
-// S_w = Q_w K^T: 8 K-steps of 16 over head_dim, both operands K-major, SW128.
-template <int HALF>
+// S_w = Q_w K^T: D / 16 K-steps of 16 over head_dim, both operands K-major,
+// SW128 (steps 4-7 in the second 64-column half, HALF bytes on).
+template <int HALF, int D>
 __device__ __forceinline__ void prefill_issue_s(uint32_t d_tmem, uint32_t q_smem,
                                                 uint32_t k_smem, uint32_t idesc) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
+  for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
     umma_ss(d_tmem, umma_desc_sw128(q_smem + off, 16, 1024),
             umma_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
@@ -218,12 +222,12 @@ __device__ __forceinline__ void prefill_p_chunks(const uint32_t (&sv)[128], uint
 // tensor-memory columns.  SOFT_REGS / PROD_REGS: the setmaxnreg split between
 // the two softmax warpgroups and every other warpgroup of the CTA.
 template <typename T, int BS, uint32_t SOFT_REGS = PrefillShape<T, BS>::SOFTMAX_REGS,
-          uint32_t PROD_REGS = PrefillShape<T, BS>::PRODUCER_REGS>
+          uint32_t PROD_REGS = PrefillShape<T, BS>::PRODUCER_REGS, int HEAD_DIM = 128>
 __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const PrefillParams& p,
                                              uint8_t* smem, int tile, int h, int s, int part = 0,
                                              int nparts = 1, int slot = 0) {
-  using Sh = PrefillShape<T, BS>;
+  using Sh = PrefillShape<T, BS, HEAD_DIM>;
   constexpr int D = Sh::D, BM = Sh::BM, BN = Sh::BN, NQ = Sh::NQ, NS = Sh::NSTAGE;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::BAR_OFF);
@@ -314,8 +318,8 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
       mbar_arrive_expect_tx(q_full, NQ * Sh::TILE);
     }
     __syncwarp();
-    if (lane < 2 * NQ) {  // lane -> (Q tile, 64-column half)
-      const int w = lane >> 1, hf = lane & 1;
+    if (lane < Sh::NH * NQ) {  // lane -> (Q tile, 64-column half)
+      const int w = lane / Sh::NH, hf = lane % Sh::NH;
       tma_load_2d(smem + Sh::Q_OFF + w * Sh::TILE + hf * Sh::HALF, tm_q, h * D + hf * 64,
                   q0 + i0 + w * BM, q_full, pol_q);
     }
@@ -331,8 +335,8 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
           phys = 0;
         }
       }
-      // lane l issues the box of block l / 2, 64-column half l % 2
-      const int ph = __shfl_sync(0xffffffffu, phys, (lane >> 1) & 31);
+      // lane l issues the box of block l / NH, 64-column half l % NH
+      const int ph = __shfl_sync(0xffffffffu, phys, (lane / Sh::NH) & 31);
       const int row = (ph * p.num_kv_heads + kvh) * BS;
       const uint32_t bytes = (uint32_t)nb * BS * D * 2;
 #pragma unroll
@@ -344,10 +348,11 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
           if (ok) mbar_arrive_expect_tx(&ring_full[st], bytes);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // gave up: load nothing more
-        if (lane < 2 * nb) {
-          tma_load_2d(smem + Sh::RING_OFF + st * Sh::TILE + (lane & 1) * Sh::HALF +
-                          (lane >> 1) * BS * 128,
-                      kv == 0 ? tm_k : tm_v, (lane & 1) * 64, row, &ring_full[st], pol_kv);
+        if (lane < Sh::NH * nb) {
+          const int hf = lane % Sh::NH;
+          tma_load_2d(smem + Sh::RING_OFF + st * Sh::TILE + hf * Sh::HALF +
+                          (lane / Sh::NH) * BS * 128,
+                      kv == 0 ? tm_k : tm_v, hf * 64, row, &ring_full[st], pol_kv);
         }
         armed = item + 1;
       }
@@ -356,15 +361,15 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     // ------------------------------------------------------------ MMA warp
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_f16(128, 128, kBf16, false, false);
-      constexpr uint32_t idesc_pv = umma_idesc_f16(128, 128, kBf16, false, true);
+      constexpr uint32_t idesc_pv = umma_idesc_f16(128, D, kBf16, false, true);
       const uint32_t sq = smem_u32(smem + Sh::Q_OFF);
       const uint32_t ring = smem_u32(smem + Sh::RING_OFF);
       bool alive = mbar_wait(q_full, 0, abort) && mbar_wait(&ring_full[0], 0, abort);  // Q, K_0
       if (alive) {
         tc_fence_after();
-        prefill_issue_s<Sh::HALF>(tmem, sq, ring, idesc_qk);
+        prefill_issue_s<Sh::HALF, D>(tmem, sq, ring, idesc_qk);
         umma_commit(&s_full[0]);
-        prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring, idesc_qk);
+        prefill_issue_s<Sh::HALF, D>(tmem + 128, sq + Sh::TILE, ring, idesc_qk);
         umma_commit(&s_full[1]);
         umma_commit(&ring_empty[0]);
       }
@@ -388,7 +393,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
         prefill_issue_pv<Sh::HALF, 4, 8>(tmem + 256, tmem, ring + st_v * Sh::TILE, idesc_pv,
                                          false);
         if (more) {
-          prefill_issue_s<Sh::HALF>(tmem, sq, ring + st_k * Sh::TILE, idesc_qk);
+          prefill_issue_s<Sh::HALF, D>(tmem, sq, ring + st_k * Sh::TILE, idesc_qk);
           umma_commit(&s_full[0]);
         } else {
           umma_commit(&o_final[0]);
@@ -404,7 +409,7 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
                                          idesc_pv, false);
         umma_commit(&ring_empty[st_v]);
         if (more) {
-          prefill_issue_s<Sh::HALF>(tmem + 128, sq + Sh::TILE, ring + st_k * Sh::TILE, idesc_qk);
+          prefill_issue_s<Sh::HALF, D>(tmem + 128, sq + Sh::TILE, ring + st_k * Sh::TILE, idesc_qk);
           umma_commit(&s_full[1]);
           umma_commit(&ring_empty[st_k]);
         } else {
@@ -440,8 +445,9 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
         if (alive) alive = mbar_wait(&ring_full[st_v], (it_v / NS) & 1, abort);
         const int first = L - kbase;
         uint8_t* vs = smem + Sh::RING_OFF + st_v * Sh::TILE;
-        for (int idx = r; idx < (BN - first) * 16; idx += 128) {
-          const int vr = first + idx / 16, ch = idx % 16;
+        constexpr int CH = D / 8;  // 16-byte chunks per row
+        for (int idx = r; idx < (BN - first) * CH; idx += 128) {
+          const int vr = first + idx / CH, ch = idx % CH;
           *reinterpret_cast<uint4*>(vs + (ch >> 3) * Sh::HALF + vr * 128 + (ch & 7) * 16) =
               make_uint4(0, 0, 0, 0);
         }
@@ -525,8 +531,10 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
     uint32_t ov[D];
     tmem_ld32_at<0>(t_o, ov);
     tmem_ld32_at<32>(t_o + 32, ov);
-    tmem_ld32_at<64>(t_o + 64, ov);
-    tmem_ld32_at<96>(t_o + 96, ov);
+    if constexpr (D == 128) {
+      tmem_ld32_at<64>(t_o + 64, ov);
+      tmem_ld32_at<96>(t_o + 96, ov);
+    }
     tmem_wait_ld();
     if (nparts == 1) {
       if (row < n) {
@@ -575,8 +583,8 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   }
 }
 
-template <typename T, int BS>
-__global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
+template <typename T, int BS, int D>
+__global__ void __launch_bounds__(PrefillShape<T, BS, D>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
@@ -595,7 +603,8 @@ __global__ void __launch_bounds__(PrefillShape<T, BS>::THREADS, 1)
   const int tile = unit % p.tiles_per_seq;
   const int h = (unit / p.tiles_per_seq) % p.num_q_heads;
   const int s = unit / (p.tiles_per_seq * p.num_q_heads);
-  prefill_tile<T, BS>(&tm_q, &tm_k, &tm_v, p, smem, tile, h, s, part, nparts, slot);
+  prefill_tile<T, BS, PrefillShape<T, BS, D>::SOFTMAX_REGS, PrefillShape<T, BS, D>::PRODUCER_REGS,
+               D>(&tm_q, &tm_k, &tm_v, p, smem, tile, h, s, part, nparts, slot);
 }
 
 }  // namespace pa

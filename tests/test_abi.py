@@ -124,7 +124,7 @@ def test_prefill_rejects_bad_arguments(lib):
     assert call(cu=None) == pa.PA_ERR_INVALID_ARG
     assert call(mc=16 * 16) == pa.PA_ERR_INVALID_ARG            # context fills the table
     assert call(hq=3, hkv=2) == pa.PA_ERR_INVALID_ARG
-    assert call(d=64) == pa.PA_ERR_UNSUPPORTED
+    assert call(d=96) == pa.PA_ERR_UNSUPPORTED                   # head_dim 64 or 128
     assert call(bs=64, mb=4) == pa.PA_ERR_UNSUPPORTED
     assert call(tq=0) == pa.PA_OK
 

@@ -1,8 +1,9 @@
 """pa_prefill_chunk (tcgen05) against the fp64 oracle: ragged chunks and
-contexts across several 128-row / 128-key tiles, both block sizes and both
-16-bit types, NaN in unused slots, the full-size 8 x 512-token chunk
-workload on sampled rows, and bit-identical output under a relabelling of the
-physical blocks, with and without the key-range split of the last wave."""
+contexts across several 128-row / 128-key tiles, both block sizes, both
+16-bit types and head_dim 128 and 64, NaN in unused slots, the full-size
+8 x 512-token chunk workload on sampled rows, and bit-identical output under a
+relabelling of the physical blocks, with and without the key-range split of
+the last wave."""
 import dataclasses
 
 import numpy as np
@@ -58,6 +59,37 @@ def test_ragged_chunks_match_oracle(B, dtype, hq, hkv, split_tail):
     oracle_scatter(p)
     ref, _ = reference(p)
     assert max_err(out, ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("B", [16, 32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("split_tail", [True, False])
+def test_head_dim_64_matches_oracle(B, dtype, split_tail):
+    # the same ragged batch at head_dim 64 (one 64-column half per row, 8-stage
+    # ring, PV products N = 64): 2 tiles x 8 heads x 5 sequences = 80 units
+    ctx = [0, 5, 40, 200, 129]
+    qn = [1, 130, 7, 300, 256]
+    p = synth.chunked_prefill(seed=B + 64, block_size=B, hq=8, hkv=2, d=64, dtype=dtype,
+                              ctx_lens=ctx, q_lens=qn)
+    out = run_prefill(p, split_tail)
+    oracle_scatter(p)
+    ref, _ = reference(p)
+    assert torch.isfinite(out.float()).all()
+    assert max_err(out, ref) <= TOL[dtype]
+
+
+def test_head_dim_64_long_context_split_tail():
+    # one sequence over 8192 + 512 keys at head_dim 64: 16 units, each split
+    # four ways, so the partial rows (D / 4 float4 per row) and their combine
+    # run at head_dim 64 too
+    p = synth.chunked_prefill(seed=13, block_size=16, num_seqs=1, hq=8, hkv=2, d=64)
+    a = run_prefill(p, split_tail=True)
+    b = run_prefill(p, split_tail=False)
+    oracle_scatter(p)
+    rows = [0, 1, 127, 128, 255, 256, 300, 511]
+    ref, _ = reference(p, rows=rows)
+    assert max_err(a[rows], ref[rows]) <= TOL[p.dtype]
+    assert max_err(b[rows], ref[rows]) <= TOL[p.dtype]
 
 
 def test_nan_in_unused_slots_does_not_leak():
@@ -140,11 +172,12 @@ RELABEL_CASES = {
 @pytest.mark.parametrize("case", sorted(RELABEL_CASES))
 @pytest.mark.parametrize("B", [16, 32])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-def test_prefill_bit_identical_under_block_relabelling(case, B, dtype):
+@pytest.mark.parametrize("d", [128, 64])
+def test_prefill_bit_identical_under_block_relabelling(case, B, dtype, d):
     # The result may depend only on logical positions, never on where the
     # blocks sit in the pool ("vLLM PagedAttention Deep Dive", "PagedAttention
     # Mechanism"): with and without the key-range split of the last wave.
-    p = synth.chunked_prefill(seed=31 + B, block_size=B, dtype=dtype, d=128,
+    p = synth.chunked_prefill(seed=31 + B, block_size=B, dtype=dtype, d=d,
                               **RELABEL_CASES[case])
     moved = _relabelled(p, seed=5 + B)
     for split_tail in (True, False):
