@@ -481,6 +481,91 @@ __device__ __forceinline__ int produce_item(const CUtensorMap* tm_k, const CUten
 // Positions >= L (the end of the item's tokens) are masked and their V rows
 // zeroed.  With HP > 1, tile rows [h*TT, (h+1)*TT) hold head h of the pack
 // and only query columns [h*G, (h+1)*G) see them.
+// consume_block for a stage of two packed KV heads (rows 0-15: head 0's
+// tokens, rows 16-31: head 1's, the same 16 positions from t_lo - r4): query
+// column g belongs to head g / G (g >= 2G: padding), so each column uses the
+// scores of one sub-tile only and one online-softmax pass (one max
+// reduction, four exponentials per lane) serves both; P of each sub-tile keeps
+// only its head's columns.  The per-column arithmetic is that of two
+// separate passes (the other pass only adds zeros), so the result is the same
+// bit for bit.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void consume_packed_pair(
+    float (&o)[Tiles::D / 16][NT][4], float (&m_run)[NT][2], float (&l_run)[NT][2],
+    const uint32_t (&qf)[Tiles::D / 16][NT][2], const uint8_t* sk, const uint8_t* sv, int t_lo,
+    int L, float scale_log2, int lane, int G) {
+  using MmaT = typename Tiles::MmaT;
+  constexpr int D = Tiles::D;
+  const int c4 = lane & 3;
+  float sacc[2][NT][4];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[hh][nt][e] = 0.f;
+  Tiles::template qk<NT>(sacc[0], sk, 0, qf, lane);
+  Tiles::template qk<NT>(sacc[1], sk, 1, qf, lane);
+  const bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+  int head[NT][2];
+  float sl[NT][2], sh[NT][2], alpha[NT][2];
+  bool raise = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hc = (nt * 8 + 2 * c4 + j) / G;
+      head[nt][j] = hc;
+      const float lo = hc == 0 ? sacc[0][nt][j] : sacc[1][nt][j];
+      const float hi = hc == 0 ? sacc[0][nt][j + 2] : sacc[1][nt][j + 2];
+      sl[nt][j] = ok_lo && hc < 2 ? lo * scale_log2 : -INFINITY;
+      sh[nt][j] = ok_hi && hc < 2 ? hi * scale_log2 : -INFINITY;
+      float mx = fmaxf(sl[nt][j], sh[nt][j]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      alpha[nt][j] = 1.f;
+      if (mx > m_run[nt][j] + 8.f) {
+        alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);
+        m_run[nt][j] = mx;
+        raise = true;
+      }
+    }
+  if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        l_run[nt][j] *= alpha[nt][j];
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt) {
+          o[dt][nt][j] *= alpha[nt][j];
+          o[dt][nt][j + 2] *= alpha[nt][j];
+        }
+      }
+  }
+  uint32_t pb[2][NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float pv[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float m_use = m_run[nt][j] == -INFINITY ? 0.f : m_run[nt][j];
+      pv[j] = ex2_approx(sl[nt][j] - m_use);
+      pv[j + 2] = ex2_approx(sh[nt][j] - m_use);
+      l_run[nt][j] += pv[j] + pv[j + 2];
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const bool m0 = head[nt][0] == hh, m1 = head[nt][1] == hh;
+      pb[hh][nt][0] = movmatrix_trans(MmaOp<MmaT>::pack(m0 ? pv[0] : 0.f, m1 ? pv[1] : 0.f));
+      pb[hh][nt][1] = movmatrix_trans(MmaOp<MmaT>::pack(m0 ? pv[2] : 0.f, m1 ? pv[3] : 0.f));
+    }
+  }
+  Tiles::template pv<NT>(o, sv, 0, pb[0], lane);
+  Tiles::template pv<NT>(o, sv, 1, pb[1], lane);
+}
+
 template <class Tiles, int BS, int NT>
 __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
                                               float (&m_run)[NT][2], float (&l_run)[NT][2],
@@ -504,6 +589,12 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
           make_uint4(0, 0, 0, 0);
     }
     __syncwarp();
+  }
+  if constexpr (HP == 2) {
+    consume_packed_pair<Tiles, BS, NT>(o, m_run, l_run, qf, sk, sv, tok_blk + r4, L, scale_log2,
+                                       lane, G);
+    if (valid < TT) fence_proxy_async_smem();
+    return;
   }
 #pragma unroll
   for (int mt = 0; mt < Shape::ROWS / 16; ++mt) {
