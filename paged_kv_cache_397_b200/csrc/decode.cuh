@@ -481,6 +481,49 @@ __device__ __forceinline__ int produce_item(const CUtensorMap* tm_k, const CUten
 // Positions >= L (the end of the item's tokens) are masked and their V rows
 // zeroed.  With HP > 1, tile rows [h*TT, (h+1)*TT) hold head h of the pack
 // and only query columns [h*G, (h+1)*G) see them.
+// Running max of the online softmax, per query column (the 8 lanes with the
+// same lane % 4 hold a column's 16 rows): raised only when a sub-tile's column
+// max exceeds it by more than 8 (log2 units), so P <= 2^8 stays in 16-bit
+// range and O is rescaled rarely (the stale max cancels in O / l).
+// running_max_may_rise: one warp vote on whether any lane holds a score above
+// its column's m_run + 8 — when none does, no column max can exceed it either,
+// and the per-column shuffle reductions are skipped (the common case).
+template <int NT>
+__device__ __forceinline__ bool running_max_may_rise(const float (&sl)[NT][2],
+                                                     const float (&sh)[NT][2],
+                                                     const float (&m_run)[NT][2]) {
+  bool above = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) above |= fmaxf(sl[nt][j], sh[nt][j]) > m_run[nt][j] + 8.f;
+  return __any_sync(0xffffffffu, above);
+}
+// The column maxima (3 shuffles each) and the raise; alpha = 2^(old - new)
+// for raised columns (0 when the old max was -inf).  Returns this lane's
+// "some column rose".
+template <int NT>
+__device__ __forceinline__ bool raise_running_max(const float (&sl)[NT][2],
+                                                  const float (&sh)[NT][2], float (&m_run)[NT][2],
+                                                  float (&alpha)[NT][2]) {
+  bool raise = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float mx = fmaxf(sl[nt][j], sh[nt][j]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      if (mx > m_run[nt][j] + 8.f) {
+        alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);
+        m_run[nt][j] = mx;
+        raise = true;
+      }
+    }
+  return raise;
+}
+
 // consume_block for a stage of two packed KV heads (rows 0-15: head 0's
 // tokens, rows 16-31: head 1's, the same 16 positions from t_lo - r4): query
 // column g belongs to head g / G (g >= 2G: padding), so each column uses the
@@ -520,17 +563,10 @@ __device__ __forceinline__ void consume_packed_pair(
       const float hi = hc == 0 ? sacc[0][nt][j + 2] : sacc[1][nt][j + 2];
       sl[nt][j] = ok_lo && hc < 2 ? lo * scale_log2 : -INFINITY;
       sh[nt][j] = ok_hi && hc < 2 ? hi * scale_log2 : -INFINITY;
-      float mx = fmaxf(sl[nt][j], sh[nt][j]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       alpha[nt][j] = 1.f;
-      if (mx > m_run[nt][j] + 8.f) {
-        alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);
-        m_run[nt][j] = mx;
-        raise = true;
-      }
     }
+  if (running_max_may_rise<NT>(sl, sh, m_run))
+    raise = raise_running_max<NT>(sl, sh, m_run, alpha);
   if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -613,9 +649,7 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
 #pragma unroll
       for (int j = 0; j < 2; ++j)
         col_ok[nt][j] = HP == 1 || (nt * 8 + 2 * c4 + j) / G == (mt * 16) / TT;
-    // The running max m_run is raised only when a sub-tile's max exceeds
-    // it by more than 8 (log2 units), so P <= 2^8 stays in 16-bit range and
-    // O is rescaled rarely; the stale max cancels in O / l.
+    // running max: see running_max_may_rise / raise_running_max
     uint32_t pb[NT][2];
     float sl[NT][2], sh[NT][2], alpha[NT][2];
     bool raise = false;
@@ -625,17 +659,10 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
       for (int j = 0; j < 2; ++j) {
         sl[nt][j] = ok_lo && col_ok[nt][j] ? sacc[nt][j] * scale_log2 : -INFINITY;
         sh[nt][j] = ok_hi && col_ok[nt][j] ? sacc[nt][j + 2] * scale_log2 : -INFINITY;
-        float mx = fmaxf(sl[nt][j], sh[nt][j]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         alpha[nt][j] = 1.f;
-        if (mx > m_run[nt][j] + 8.f) {
-          alpha[nt][j] = ex2_approx(m_run[nt][j] - mx);  // 0 when m_run is -inf
-          m_run[nt][j] = mx;
-          raise = true;
-        }
       }
+    if (running_max_may_rise<NT>(sl, sh, m_run))
+      raise = raise_running_max<NT>(sl, sh, m_run, alpha);
     if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
