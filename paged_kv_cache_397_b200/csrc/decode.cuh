@@ -104,7 +104,7 @@ struct HalfTiles {
   static constexpr int NS = BS == 16 ? 8 : 4;        // ring depth
   static constexpr int NW = 4;                       // consumer warps per CTA
   // resident CTAs per SM to plan registers for, by query n-tiles per CTA
-  static constexpr int min_ctas(int) { return 2; }
+  static constexpr int min_ctas(int nt) { return nt == 1 ? 3 : 2; }
   static constexpr int ZERO_CHUNKS_PER_ROW = BOXES * 8;
 
   // K and V of the cache block at pool row `row` into block slot u (always 0)
@@ -859,10 +859,18 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   const int blk0 = part * p.part_blocks;
   const int nblk = min(p.part_blocks, nblk_seq - blk0);  // 0 only when L == 0
 
+  // The producer warp issues the first NS ring positions; after that the
+  // consumer warp that finishes position i issues position i + NS into the
+  // same stage itself (NS is a multiple of NW, so that position is its own):
+  // a stage is refilled the moment it is free, never behind another warp's
+  // slower stage.  last_fill[st] is the last position issued on stage st
+  // (for the drain after an abort); the empty barriers are not used here.
+  const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
+  int* last_fill = reinterpret_cast<int*>(empty_bar);
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
+      last_fill[i] = i < nstages ? i : -1;
     }
     *abort = 0;
     fence_barrier_init();
@@ -883,13 +891,17 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
       else if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
         p.slot_out[s] = -1;
     }
-    bool alive = true;
-    const int armed = produce_item<Tiles, BS, NT>(
-        tm_k, tm_v, p, smem, full_bar, empty_bar,
-        p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, blk0, nblk, 0, lane,
-        l2_policy_evict_first(), alive, abort);
+    bool alive = true;  // positions < NS wait for nothing: all of them are issued
+    produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar,
+                                p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, blk0,
+                                min(nblk, NS * Shape::SB), 0, lane, l2_policy_evict_first(),
+                                alive, abort);
     named_barrier(bar_all, Shape::THREADS);  // the consumers are done
-    if (*abort && lane == 0) drain_ring<NS>(full_bar, armed);
+    if (*abort && lane == 0) {
+      // a wait gave up: let every load still in flight land before the CTA ends
+      for (int st = 0; st < NS; ++st)
+        if (last_fill[st] >= 0) mbar_drain(&full_bar[st], (last_fill[st] / NS) & 1);
+    }
     return;
   }
 
@@ -903,9 +915,14 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   float m_run[NT][2], l_run[NT][2];
   float o[D / 16][NT][4];
   reset_state<Tiles, NT>(o, m_run, l_run);
-  const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
   // a stage may reach past the item's last block (into the next partition)
   const int L_end = min(L, (blk0 + nblk) * BS);
+  const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+  const uint64_t policy = l2_policy_evict_first();
+  // Block ids of this warp's refills: lane l holds the blocks of the warp's
+  // (kw + l)-th position (position warp + NW * (kw + l)), fetched 32 at a time.
+  int ids[Shape::SB];
+  int kw = -32;
   bool alive = true;
   for (int i = warp; i < nstages; i += NW) {
     const int st = i % NS;
@@ -916,7 +933,44 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
                                  (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane,
                                  p.group);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[st]);
+    const int nxt = i + NS;  // the next fill of stage st (warp-uniform test)
+    if (nxt < nstages) {
+      const int k = (nxt - warp) / NW;
+      if (k >= kw + 32) {
+        kw = k;
+#pragma unroll
+        for (int u = 0; u < Shape::SB; ++u) {
+          const int b = (warp + NW * (k + lane)) * Shape::SB + u;
+          int id = 0;
+          if (b < nblk) {
+            id = __ldg(bt + b);
+            if (id < 0 || id >= p.num_blocks) {
+              record_error(PA_DEVERR_BLOCK_RANGE);
+              id = 0;
+            }
+          }
+          ids[u] = id;
+        }
+      }
+      int ph[Shape::SB];
+#pragma unroll
+      for (int u = 0; u < Shape::SB; ++u) ph[u] = __shfl_sync(0xffffffffu, ids[u], k - kw);
+      if (lane == 0 && alive) {
+        // this warp's reads of the stage are done (__syncwarp above); order
+        // them before the async-proxy writes that refill it
+        fence_proxy_async_smem();
+        const int nb = min(Shape::SB, nblk - nxt * Shape::SB);
+        mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
+        uint8_t* sk = smem + st * Shape::STAGE_BYTES;
+#pragma unroll
+        for (int u = 0; u < Shape::SB; ++u)
+          if (u < nb)
+            Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
+                         (ph[u] * p.num_kv_heads + kvh * Shape::HP) * BS, u, &full_bar[st],
+                         policy);
+        last_fill[st] = nxt;
+      }
+    }
   }
   // the merge area aliases the ring: merge_item's opening barrier waits for
   // every consumer to finish reading it (after an abort a late load may still
