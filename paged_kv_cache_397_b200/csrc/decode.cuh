@@ -629,68 +629,67 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
   if constexpr (HP == 2) {
     consume_packed_pair<Tiles, BS, NT>(o, m_run, l_run, qf, sk, sv, tok_blk + r4, L, scale_log2,
                                        lane, G);
-    if (valid < TT) fence_proxy_async_smem();
-    return;
-  }
+  } else {
 #pragma unroll
-  for (int mt = 0; mt < Shape::ROWS / 16; ++mt) {
-    float sacc[NT][4];
+    for (int mt = 0; mt < Shape::ROWS / 16; ++mt) {
+      float sacc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-    Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
-    // online softmax over this sub-tile's 16 rows (tokens of one head)
-    const int t_lo = tok_blk + (mt * 16) % TT + r4;
-    bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
-    bool col_ok[NT][2];
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+      Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
+      // online softmax over this sub-tile's 16 rows (tokens of one head)
+      const int t_lo = tok_blk + (mt * 16) % TT + r4;
+      bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+      bool col_ok[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
-        col_ok[nt][j] = HP == 1 || (nt * 8 + 2 * c4 + j) / G == (mt * 16) / TT;
-    // running max: see running_max_may_rise / raise_running_max
-    uint32_t pb[NT][2];
-    float sl[NT][2], sh[NT][2], alpha[NT][2];
-    bool raise = false;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        sl[nt][j] = ok_lo && col_ok[nt][j] ? sacc[nt][j] * scale_log2 : -INFINITY;
-        sh[nt][j] = ok_hi && col_ok[nt][j] ? sacc[nt][j + 2] * scale_log2 : -INFINITY;
-        alpha[nt][j] = 1.f;
-      }
-    if (running_max_may_rise<NT>(sl, sh, m_run))
-      raise = raise_running_max<NT>(sl, sh, m_run, alpha);
-    if (__any_sync(0xffffffffu, raise)) {
+        for (int j = 0; j < 2; ++j)
+          col_ok[nt][j] = HP == 1 || (nt * 8 + 2 * c4 + j) / G == (mt * 16) / TT;
+      // running max: see running_max_may_rise / raise_running_max
+      uint32_t pb[NT][2];
+      float sl[NT][2], sh[NT][2], alpha[NT][2];
+      bool raise = false;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          l_run[nt][j] *= alpha[nt][j];
-#pragma unroll
-          for (int dt = 0; dt < D / 16; ++dt) {
-            o[dt][nt][j] *= alpha[nt][j];
-            o[dt][nt][j + 2] *= alpha[nt][j];
-          }
+          sl[nt][j] = ok_lo && col_ok[nt][j] ? sacc[nt][j] * scale_log2 : -INFINITY;
+          sh[nt][j] = ok_hi && col_ok[nt][j] ? sacc[nt][j + 2] * scale_log2 : -INFINITY;
+          alpha[nt][j] = 1.f;
         }
-    }
+      if (running_max_may_rise<NT>(sl, sh, m_run))
+        raise = raise_running_max<NT>(sl, sh, m_run, alpha);
+      if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float pv[4];
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float m_use = m_run[nt][j] == -INFINITY ? 0.f : m_run[nt][j];
-        pv[j] = ex2_approx(sl[nt][j] - m_use);
-        pv[j + 2] = ex2_approx(sh[nt][j] - m_use);
-        l_run[nt][j] += pv[j] + pv[j + 2];
+          for (int j = 0; j < 2; ++j) {
+            l_run[nt][j] *= alpha[nt][j];
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+              o[dt][nt][j] *= alpha[nt][j];
+              o[dt][nt][j + 2] *= alpha[nt][j];
+            }
+          }
       }
-      // accumulator rows t / t+8, cols (g, g+1) -> B-operand layout of P^T
-      pb[nt][0] = movmatrix_trans(MmaOp<MmaT>::pack(pv[0], pv[1]));
-      pb[nt][1] = movmatrix_trans(MmaOp<MmaT>::pack(pv[2], pv[3]));
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float pv[4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float m_use = m_run[nt][j] == -INFINITY ? 0.f : m_run[nt][j];
+          pv[j] = ex2_approx(sl[nt][j] - m_use);
+          pv[j + 2] = ex2_approx(sh[nt][j] - m_use);
+          l_run[nt][j] += pv[j] + pv[j + 2];
+        }
+        // accumulator rows t / t+8, cols (g, g+1) -> B-operand layout of P^T
+        pb[nt][0] = movmatrix_trans(MmaOp<MmaT>::pack(pv[0], pv[1]));
+        pb[nt][1] = movmatrix_trans(MmaOp<MmaT>::pack(pv[2], pv[3]));
+      }
+      Tiles::template pv<NT>(o, sv, mt, pb, lane);
     }
-    Tiles::template pv<NT>(o, sv, mt, pb, lane);
   }
   if (valid < TT) fence_proxy_async_smem();  // our zero stores precede the next TMA write
 }
@@ -832,6 +831,107 @@ __device__ __forceinline__ void append_new_token(const DecodeParams& p, int s, i
   __syncwarp();
 }
 
+// Ring protocol of one work item.  The producer warp issues the first NS ring
+// positions (item_ring_fill); after that the consumer warp that finishes
+// position i issues position i + NS into the same stage itself (NS is a
+// multiple of NW, so that position is its own), so a stage is refilled the
+// moment it is free, never behind another warp's slower stage.
+// last_fill[st] (shared) is the last position issued on stage st, for the
+// drain after an abort (item_ring_drain); the empty barriers are not used.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void item_ring_init(uint64_t* full_bar, int* last_fill, int nstages) {
+  constexpr int NS = DecodeShape<Tiles, BS, NT>::NS;
+  for (int i = 0; i < NS; ++i) {
+    mbar_init(&full_bar[i], 1);
+    last_fill[i] = i < nstages ? i : -1;
+  }
+}
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void item_ring_fill(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                               const DecodeParams& p, uint8_t* smem,
+                                               uint64_t* full_bar, uint64_t* empty_bar,
+                                               const int32_t* table, int kvh, int blk0, int nblk,
+                                               int lane, uint64_t policy, volatile int* abort) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  bool alive = true;  // positions < NS wait for nothing: all of them are issued
+  produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar, table, kvh, blk0,
+                              min(nblk, Shape::NS * Shape::SB), 0, lane, policy, alive, abort);
+}
+// After an abort (one thread): let every load still in flight land.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void item_ring_drain(uint64_t* full_bar, const int* last_fill) {
+  constexpr int NS = DecodeShape<Tiles, BS, NT>::NS;
+  for (int st = 0; st < NS; ++st)
+    if (last_fill[st] >= 0) mbar_drain(&full_bar[st], (last_fill[st] / NS) & 1);
+}
+
+// Consumer side of one item (blocks blk0 .. blk0 + nblk - 1 of the table row
+// `bt`, which starts at block blk0): consume_block over the warp's ring
+// positions, each followed by the refill of its stage.  The warp's refill
+// block ids sit in a register window: lane l holds the blocks of the warp's
+// (kw + l)-th position, fetched 32 positions at a time.
+template <class Tiles, int BS, int NT>
+__device__ __forceinline__ void consume_item(
+    float (&o)[Tiles::D / 16][NT][4], float (&m_run)[NT][2], float (&l_run)[NT][2],
+    const uint32_t (&qf)[Tiles::D / 16][NT][2], const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+    const DecodeParams& p, uint8_t* smem, uint64_t* full_bar, int* last_fill,
+    const int32_t* bt, int kvh, int blk0, int nblk, int L_end, int G, uint64_t policy, int warp,
+    int lane, volatile int* abort) {
+  using Shape = DecodeShape<Tiles, BS, NT>;
+  constexpr int NW = Shape::NW, NS = Shape::NS, SB = Shape::SB;
+  const int nstages = (nblk + SB - 1) / SB;
+  int ids[SB];
+  int kw = -32;
+  bool alive = true;
+  for (int i = warp; i < nstages; i += NW) {
+    const int st = i % NS;
+    // after a wait gave up the warp still runs through its (garbage) stages,
+    // every lane alike, so the .aligned loads and MMAs stay converged
+    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1, abort);
+    consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
+                                 (blk0 + i * SB) * BS, L_end, p.scale_log2, lane, G);
+    __syncwarp();
+    const int nxt = i + NS;  // the next fill of stage st (warp-uniform test)
+    if (nxt < nstages) {
+      const int k = (nxt - warp) / NW;
+      if (k >= kw + 32) {
+        kw = k;
+#pragma unroll
+        for (int u = 0; u < SB; ++u) {
+          const int b = (warp + NW * (k + lane)) * SB + u;
+          int id = 0;
+          if (b < nblk) {
+            id = __ldg(bt + b);
+            if (id < 0 || id >= p.num_blocks) {
+              record_error(PA_DEVERR_BLOCK_RANGE);
+              id = 0;
+            }
+          }
+          ids[u] = id;
+        }
+      }
+      int ph[SB];
+#pragma unroll
+      for (int u = 0; u < SB; ++u) ph[u] = __shfl_sync(0xffffffffu, ids[u], k - kw);
+      if (lane == 0 && alive) {
+        // this warp's reads of the stage are done (__syncwarp above); order
+        // them before the async-proxy writes that refill it
+        fence_proxy_async_smem();
+        const int nb = min(SB, nblk - nxt * SB);
+        mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
+        uint8_t* sk = smem + st * Shape::STAGE_BYTES;
+#pragma unroll
+        for (int u = 0; u < SB; ++u)
+          if (u < nb)
+            Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
+                         (ph[u] * p.num_kv_heads + kvh * Shape::HP) * BS, u, &full_bar[st],
+                         policy);
+        last_fill[st] = nxt;
+      }
+    }
+  }
+}
+
 // One work item (split-KV partition `part` of KV head `kvh` of sequence `s`)
 // run by THREADS consecutive threads (`tid` 0 .. THREADS-1) that own the
 // 1024-byte aligned shared memory at `smem` (SMEM_BYTES - 1024 bytes).  They
@@ -859,19 +959,11 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   const int blk0 = part * p.part_blocks;
   const int nblk = min(p.part_blocks, nblk_seq - blk0);  // 0 only when L == 0
 
-  // The producer warp issues the first NS ring positions; after that the
-  // consumer warp that finishes position i issues position i + NS into the
-  // same stage itself (NS is a multiple of NW, so that position is its own):
-  // a stage is refilled the moment it is free, never behind another warp's
-  // slower stage.  last_fill[st] is the last position issued on stage st
-  // (for the drain after an abort); the empty barriers are not used here.
+  // ring protocol: item_ring_init; the empty barriers' memory holds last_fill
   const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
   int* last_fill = reinterpret_cast<int*>(empty_bar);
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full_bar[i], 1);
-      last_fill[i] = i < nstages ? i : -1;
-    }
+    item_ring_init<Tiles, BS, NT>(full_bar, last_fill, nstages);
     *abort = 0;
     fence_barrier_init();
   }
@@ -891,17 +983,11 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
       else if (lane == 0 && kvh == 0 && p.slot_out != nullptr)
         p.slot_out[s] = -1;
     }
-    bool alive = true;  // positions < NS wait for nothing: all of them are issued
-    produce_item<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar,
-                                p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, blk0,
-                                min(nblk, NS * Shape::SB), 0, lane, l2_policy_evict_first(),
-                                alive, abort);
+    item_ring_fill<Tiles, BS, NT>(tm_k, tm_v, p, smem, full_bar, empty_bar,
+                                  p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, blk0,
+                                  nblk, lane, l2_policy_evict_first(), abort);
     named_barrier(bar_all, Shape::THREADS);  // the consumers are done
-    if (*abort && lane == 0) {
-      // a wait gave up: let every load still in flight land before the CTA ends
-      for (int st = 0; st < NS; ++st)
-        if (last_fill[st] >= 0) mbar_drain(&full_bar[st], (last_fill[st] / NS) & 1);
-    }
+    if (*abort && lane == 0) item_ring_drain<Tiles, BS, NT>(full_bar, last_fill);
     return;
   }
 
@@ -917,61 +1003,9 @@ __device__ __forceinline__ void decode_item(const CUtensorMap* tm_k, const CUten
   reset_state<Tiles, NT>(o, m_run, l_run);
   // a stage may reach past the item's last block (into the next partition)
   const int L_end = min(L, (blk0 + nblk) * BS);
-  const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
-  const uint64_t policy = l2_policy_evict_first();
-  // Block ids of this warp's refills: lane l holds the blocks of the warp's
-  // (kw + l)-th position (position warp + NW * (kw + l)), fetched 32 at a time.
-  int ids[Shape::SB];
-  int kw = -32;
-  bool alive = true;
-  for (int i = warp; i < nstages; i += NW) {
-    const int st = i % NS;
-    // after a wait gave up the warp still runs through its (garbage) stages,
-    // every lane alike, so the .aligned loads and MMAs stay converged
-    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1, abort);
-    consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
-                                 (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane,
-                                 p.group);
-    __syncwarp();
-    const int nxt = i + NS;  // the next fill of stage st (warp-uniform test)
-    if (nxt < nstages) {
-      const int k = (nxt - warp) / NW;
-      if (k >= kw + 32) {
-        kw = k;
-#pragma unroll
-        for (int u = 0; u < Shape::SB; ++u) {
-          const int b = (warp + NW * (k + lane)) * Shape::SB + u;
-          int id = 0;
-          if (b < nblk) {
-            id = __ldg(bt + b);
-            if (id < 0 || id >= p.num_blocks) {
-              record_error(PA_DEVERR_BLOCK_RANGE);
-              id = 0;
-            }
-          }
-          ids[u] = id;
-        }
-      }
-      int ph[Shape::SB];
-#pragma unroll
-      for (int u = 0; u < Shape::SB; ++u) ph[u] = __shfl_sync(0xffffffffu, ids[u], k - kw);
-      if (lane == 0 && alive) {
-        // this warp's reads of the stage are done (__syncwarp above); order
-        // them before the async-proxy writes that refill it
-        fence_proxy_async_smem();
-        const int nb = min(Shape::SB, nblk - nxt * Shape::SB);
-        mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
-        uint8_t* sk = smem + st * Shape::STAGE_BYTES;
-#pragma unroll
-        for (int u = 0; u < Shape::SB; ++u)
-          if (u < nb)
-            Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
-                         (ph[u] * p.num_kv_heads + kvh * Shape::HP) * BS, u, &full_bar[st],
-                         policy);
-        last_fill[st] = nxt;
-      }
-    }
-  }
+  consume_item<Tiles, BS, NT>(o, m_run, l_run, qf, tm_k, tm_v, p, smem, full_bar, last_fill,
+                              p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0, kvh, blk0,
+                              nblk, L_end, p.group, l2_policy_evict_first(), warp, lane, abort);
   // the merge area aliases the ring: merge_item's opening barrier waits for
   // every consumer to finish reading it (after an abort a late load may still
   // land there; the output is garbage then, and the error word says so)
@@ -1030,11 +1064,10 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, 2>::THREADS, Tiles::min
   const int blk0 = part * p.part_blocks, nblk = p.part_blocks;
   const int L_end = (blk0 + nblk) * BS;  // every token of the partition is valid
 
+  const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
+  int* last_fill = reinterpret_cast<int*>(empty_bar);  // ring protocol: item_ring_init
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
-    }
+    item_ring_init<Tiles, BS, NT>(full_bar, last_fill, nstages);
     *abort = 0;
     fence_barrier_init();
     // every sequence must hold the whole shared partition
@@ -1053,13 +1086,11 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, 2>::THREADS, Tiles::min
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
-    bool alive = true;
     // the shared tiles are read by every group's CTA: keep them in L2
-    const int armed = produce_item<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, full_bar, empty_bar,
-                                                  p.prefix_blocks, kvh, blk0, nblk, 0, lane,
-                                                  l2_policy_evict_last(), alive, abort);
+    item_ring_fill<Tiles, BS, NT>(&tm_k, &tm_v, p, smem, full_bar, empty_bar, p.prefix_blocks,
+                                  kvh, blk0, nblk, lane, l2_policy_evict_last(), abort);
     named_barrier(0, Shape::THREADS);  // the consumers are done
-    if (*abort && lane == 0) drain_ring<NS>(full_bar, armed);
+    if (*abort && lane == 0) item_ring_drain<Tiles, BS, NT>(full_bar, last_fill);
     return;
   }
 
@@ -1077,16 +1108,9 @@ __global__ void __launch_bounds__(DecodeShape<Tiles, BS, 2>::THREADS, Tiles::min
   float m_run[NT][2], l_run[NT][2];
   float o[D / 16][NT][4];
   reset_state<Tiles, NT>(o, m_run, l_run);
-  const int nstages = (nblk + Shape::SB - 1) / Shape::SB;
-  bool alive = true;
-  for (int i = warp; i < nstages; i += NW) {
-    const int st = i % NS;
-    if (alive) alive = mbar_wait(&full_bar[st], (i / NS) & 1, abort);
-    consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
-                                 (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane, G);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[st]);
-  }
+  consume_item<Tiles, BS, NT>(o, m_run, l_run, qf, &tm_k, &tm_v, p, smem, full_bar, last_fill,
+                              p.prefix_blocks + blk0, kvh, blk0, nblk, L_end, G,
+                              l2_policy_evict_last(), warp, lane, abort);
   merge_item<Tiles, BS, NT>(
       reinterpret_cast<float*>(smem), o, m_run, l_run, p, s0, kvh, part, cols,
       [&](int sq) {
