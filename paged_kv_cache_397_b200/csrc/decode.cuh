@@ -12,12 +12,14 @@
 //    relabelling of physical blocks) and long sequences fill all 148 SMs.
 //  * GQA: the CTA reads each (block, KV head) K/V tile from HBM exactly once
 //    and applies it to all G query heads of the group.
-//  * One producer warp streams the (block, KV head) tiles — each a
-//    contiguous block_size x head_dim run of the pool — into a ring of shared
-//    memory stages with TMA (cp.async.bulk.tensor, 128-byte swizzle, boxes
-//    starting on 16-byte boundaries), completing on mbarriers.  The
-//    block-table entries of a partition are fetched once, coalesced, by the
-//    producer warp.
+//  * The (block, KV head) tiles — each a contiguous block_size x head_dim
+//    run of the pool — stream into a ring of shared-memory stages with TMA
+//    (cp.async.bulk.tensor, 128-byte swizzle, boxes starting on 16-byte
+//    boundaries), completing on mbarriers.  A producer warp issues the first
+//    ring positions (and writes the step's new token first, when the append
+//    is fused); from then on each consumer warp refills the stage it has
+//    just consumed with its own next position there, so no stage waits
+//    behind another warp's (item_ring_init / item_ring_fill / consume_item).
 //  * Four consumer warps take blocks round-robin.  Each 16-token sub-tile is
 //    a tiny GEMM pair on the warp-level tensor-core path (mma.sync m16n8k16,
 //    fp32 accumulate): S^T = K Q^T puts tokens on M and the (padded) query
