@@ -164,3 +164,20 @@ def test_out_of_pool_block_id_is_flagged_not_read():
     assert pa.pa_get_device_error() & pa.PA_DEVERR_BLOCK_RANGE
     ref = decode_reference(w, [40, 40], [0])
     assert max_err(out[:1], ref) <= TOL[w.dtype]  # the healthy sequence is unaffected
+
+
+# The decode ring holds 8 stages of one 16-token block (4 of one 32-token
+# block at block size 32); after the first ring positions of an item each
+# consumer warp refills the stage it has just consumed with its own next
+# position there.  Items of about 1, 7, 8, 9, 15, 16, 17 and 33 blocks of 16
+# tokens, one partition per sequence, cover items shorter than the ring,
+# exactly the ring, one past it, two rounds and more.
+@pytest.mark.parametrize("B", [16, 32])
+def test_ring_refill_around_the_ring_depth(B):
+    stages = [1, 7, 8, 9, 15, 16, 17, 33]
+    lens = [n * 16 - 3 for n in stages] + [n * 16 for n in stages]
+    w = synth.random_decode(61 + B, lens, dtype=torch.bfloat16, block_size=B, hq=8, hkv=2,
+                            d=128, append=False)
+    out = run_decode(w, lens, partition_tokens=1024)  # one partition per sequence
+    ref = decode_reference(w, lens, list(range(w.num_seqs)))
+    assert max_err(out, ref) <= TOL[w.dtype]

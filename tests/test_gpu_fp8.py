@@ -197,3 +197,20 @@ def test_fused_append_decode_fp8_matches_three_calls(dtype, B, hq, hkv, partitio
     w.key_cache, w.value_cache = kc_b.cpu(), vc_b.cpu()
     ref = fp8_reference(w, lens, list(range(w.num_seqs)))
     assert max_err(out_b.cpu(), ref) <= TOL[dtype]
+
+
+# The FP8 ring holds 8 stages (at block size 16 a stage is one block of two
+# packed KV heads, at 32 one block of one head); after the first 8 positions of
+# an item each consumer warp refills the stage it has just consumed.  Items of
+# about 1, 7, 8, 9, 15, 16, 17 and 33 blocks of 16 tokens, one partition per
+# sequence, cover items shorter than the ring, exactly the ring, one past it,
+# two rounds and more.
+@pytest.mark.parametrize("B", [16, 32])
+def test_fp8_ring_refill_around_the_ring_depth(B):
+    stages = [1, 7, 8, 9, 15, 16, 17, 33]
+    lens = [n * 16 - 3 for n in stages] + [n * 16 for n in stages]
+    w = synth.random_decode(71 + B, lens, dtype=torch.bfloat16, block_size=B, hq=8, hkv=2,
+                            d=128, append=False, fp8_scale=1.0 / 32)
+    out = run(w, lens, partition_tokens=1024)  # one partition per sequence
+    ref = fp8_reference(w, lens, list(range(w.num_seqs)))
+    assert max_err(out, ref) <= TOL[w.dtype]
