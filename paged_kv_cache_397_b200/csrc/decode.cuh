@@ -38,8 +38,10 @@
 //    swizzled tiles through ldmatrix / ldmatrix.trans; MMA in the cache type.
 //  * E4m3Tiles — FP8 (E4M3) caches with one scale per cache ("PagedAttention:
 //    KV cache as virtual memory", "Interviewer follow-ups": FP8 KV halves the
-//    bytes per block).  Fragments are built from 16-byte / 4-byte shared loads
-//    and converted e4m3x2 -> f16x2; MMA in fp16 (the query is rounded to fp16;
+//    bytes per block).  K fragments come from 16-byte shared loads, V^T
+//    fragments from ldmatrix .m16n16 .trans .b8 (the tokens of a sub-tile in
+//    the order that load gives, K's rows loaded in the same order), both
+//    converted e4m3x2 -> f16x2; MMA in fp16 (the query is rounded to fp16;
 //    E4M3 values are exact in fp16).  k_scale is folded into the softmax scale
 //    and v_scale multiplies the output once.
 #pragma once
@@ -206,6 +208,10 @@ struct HalfTiles {
   }
   // head-dim index of accumulator element o[dt][.][e] of lane row r4
   __device__ static int out_d(int dt, int e, int r4) { return dt * 16 + r4 + (e >> 1) * 8; }
+  // S^T accumulator rows r4 and r4 + 8 of a 16-row sub-tile hold tokens
+  // row_lo(r4) and row_lo(r4) + HI_STEP of the sub-tile
+  __device__ static int row_lo(int r4) { return r4; }
+  static constexpr int HI_STEP = 8;
 };
 
 // FP8 E4M3 cache, head_dim 128: a tile is BS rows x 128 bytes (one TMA box).
@@ -294,7 +300,7 @@ struct E4m3Tiles {
   __device__ static void qk(float (&sacc)[NT][4], const uint8_t* sk, int mt,
                             const uint32_t (&qf)[D / 16][NT][2], int lane) {
     const int c4 = lane & 3, r4 = lane >> 2;
-    const int r_lo = mt * 16 + r4, r_hi = r_lo + 8;
+    const int r_lo = mt * 16 + row_lo(r4), r_hi = r_lo + HI_STEP;
     uint4 lo[2], hi[2];  // bytes [32c, 32c+32) of rows r_lo, r_hi
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -324,39 +330,42 @@ struct E4m3Tiles {
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] += acc2[nt][e];
   }
+  // O^T += V^T P^T over a 16-token sub-tile.  ldmatrix .m16n16 .trans .b8
+  // hands lane (g = lane / 4, c = lane % 4) the bytes of head dims 16 dt + g
+  // and 16 dt + g + 8 for tokens 4c .. 4c + 3 — once converted, the A
+  // fragment of m-tile dt with the sub-tile's tokens in the order row_lo
+  // gives the S^T rows, so P^T (movmatrix of S^T) pairs with it as is.  One
+  // .x2 load covers two m-tiles (lanes 0-15 address the token rows of the
+  // first, 16-31 of the second).
   template <int NT>
   __device__ static void pv(float (&o)[D / 16][NT][4], const uint8_t* sv, int mt,
                             const uint32_t (&pb)[NT][2], int lane) {
-    const int c4 = lane & 3, r4 = lane >> 2;
-    const int t0 = mt * 16 + 2 * c4;  // token rows t0, t0+1, t0+8, t0+9
-    // bytes [16 r, 16 r + 16) of each of the four rows: word p, byte b holds
-    // head dim 16 r + 4 p + b = (m-tile 2p, row r), (2p, r+8), (2p+1, r), (2p+1, r+8)
-    const uint4 v0 = lds<uint4>(sv, t0, 16 * r4), v1 = lds<uint4>(sv, t0 + 1, 16 * r4);
-    const uint4 v8 = lds<uint4>(sv, t0 + 8, 16 * r4), v9 = lds<uint4>(sv, t0 + 9, 16 * r4);
+    const uint32_t base = smem_u32(sv);
+    const int row = mt * 16 + (lane & 15);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t w0 = p == 0 ? v0.x : p == 1 ? v0.y : p == 2 ? v0.z : v0.w;
-      const uint32_t w1 = p == 0 ? v1.x : p == 1 ? v1.y : p == 2 ? v1.z : v1.w;
-      const uint32_t w2 = p == 0 ? v8.x : p == 1 ? v8.y : p == 2 ? v8.z : v8.w;
-      const uint32_t w3 = p == 0 ? v9.x : p == 1 ? v9.y : p == 2 ? v9.z : v9.w;
-      // pair the two token rows byte by byte (contraction runs along tokens)
-      const uint32_t e01 = __byte_perm(w0, w1, 0x5140), o01 = __byte_perm(w0, w1, 0x7362);
-      const uint32_t e89 = __byte_perm(w2, w3, 0x5140), o89 = __byte_perm(w2, w3, 0x7362);
-      uint32_t ae[4], ao[4];
-      e4m3x4_to_f16x2x2(e01, ae[0], ae[1]);
-      e4m3x4_to_f16x2x2(e89, ae[2], ae[3]);
-      e4m3x4_to_f16x2x2(o01, ao[0], ao[1]);
-      e4m3x4_to_f16x2x2(o89, ao[2], ao[3]);
+    for (int dt = 0; dt < D / 16; dt += 2) {
+      const uint32_t addr = sw128(base, row, 16 * (dt + (lane >> 4)));
+      uint32_t r[4];
+      asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                   : "r"(addr));
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        MmaOp<MmaT>::run(o[2 * p][nt], ae, pb[nt][0], pb[nt][1]);
-        MmaOp<MmaT>::run(o[2 * p + 1][nt], ao, pb[nt][0], pb[nt][1]);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[4];
+        e4m3x4_to_f16x2x2(r[2 * h], a[0], a[2]);      // head dim 16 (dt + h) + g
+        e4m3x4_to_f16x2x2(r[2 * h + 1], a[1], a[3]);  // head dim 16 (dt + h) + g + 8
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) MmaOp<MmaT>::run(o[dt + h][nt], a, pb[nt][0], pb[nt][1]);
       }
     }
   }
-  __device__ static int out_d(int dt, int e, int r4) {
-    return 16 * r4 + 4 * (dt >> 1) + 2 * (dt & 1) + (e >> 1);
-  }
+  __device__ static int out_d(int dt, int e, int r4) { return dt * 16 + r4 + (e >> 1) * 8; }
+  // S^T accumulator rows r4 and r4 + 8 of a 16-row sub-tile hold tokens
+  // row_lo(r4) and row_lo(r4) + HI_STEP of the sub-tile: 0 1 4 5 8 9 12 13
+  // and 2 3 6 7 10 11 14 15 (qk loads K's rows in that order), the token
+  // order of pv's fragments
+  __device__ static int row_lo(int r4) { return 4 * (r4 >> 1) + (r4 & 1); }
+  static constexpr int HI_STEP = 2;
 };
 
 template <typename T, int BS, int HP_>
@@ -527,7 +536,8 @@ __device__ __forceinline__ bool raise_running_max(const float (&sl)[NT][2],
 }
 
 // consume_block for a stage of two packed KV heads (rows 0-15: head 0's
-// tokens, rows 16-31: head 1's, the same 16 positions from t_lo - r4): query
+// tokens, rows 16-31: head 1's, the same 16 positions; t_lo is the position
+// of this lane's S^T accumulator row, Tiles::row_lo): query
 // column g belongs to head g / G (g >= 2G: padding), so each column uses the
 // scores of one sub-tile only and one online-softmax pass (one max
 // reduction, four exponentials per lane) serves both; P of each sub-tile keeps
@@ -551,7 +561,7 @@ __device__ __forceinline__ void consume_packed_pair(
       for (int e = 0; e < 4; ++e) sacc[hh][nt][e] = 0.f;
   Tiles::template qk<NT>(sacc[0], sk, 0, qf, lane);
   Tiles::template qk<NT>(sacc[1], sk, 1, qf, lane);
-  const bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+  const bool ok_lo = t_lo < L, ok_hi = t_lo + Tiles::HI_STEP < L;
   int head[NT][2];
   float sl[NT][2], sh[NT][2], alpha[NT][2];
   bool raise = false;
@@ -629,8 +639,8 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
     __syncwarp();
   }
   if constexpr (HP == 2) {
-    consume_packed_pair<Tiles, BS, NT>(o, m_run, l_run, qf, sk, sv, tok_blk + r4, L, scale_log2,
-                                       lane, G);
+    consume_packed_pair<Tiles, BS, NT>(o, m_run, l_run, qf, sk, sv, tok_blk + Tiles::row_lo(r4),
+                                       L, scale_log2, lane, G);
   } else {
 #pragma unroll
     for (int mt = 0; mt < Shape::ROWS / 16; ++mt) {
@@ -641,8 +651,8 @@ __device__ __forceinline__ void consume_block(float (&o)[Tiles::D / 16][NT][4],
         for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
       Tiles::template qk<NT>(sacc, sk, mt, qf, lane);
       // online softmax over this sub-tile's 16 rows (tokens of one head)
-      const int t_lo = tok_blk + (mt * 16) % TT + r4;
-      bool ok_lo = t_lo < L, ok_hi = t_lo + 8 < L;
+      const int t_lo = tok_blk + (mt * 16) % TT + Tiles::row_lo(r4);
+      bool ok_lo = t_lo < L, ok_hi = t_lo + Tiles::HI_STEP < L;
       bool col_ok[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
