@@ -22,8 +22,12 @@
 //    one TMA ring without draining it between items; the consumers process
 //    each item exactly as pa_decode's CTA does (same warp for each block, same
 //    merge order), so the results are bit-identical to pa_decode.
-// The hardware hands out CTAs in launch order, so the long compute-bound
-// prefill tiles start first; decode workers start on the SMs the prefill tail
+// The grid runs as clusters of two CTAs, which share a TPC (the two SMs of a
+// tcgen05 CTA pair), and both CTAs of a cluster do the same kind of work: on
+// B200 a prefill tile whose TPC partner SM ran decode workers was measured
+// at about half speed, so a TPC runs two prefill tiles or two decode CTAs,
+// never one of each.  The hardware hands out clusters in launch order, so
+// the long compute-bound prefill tiles start first; decode workers start on the SMs the prefill tail
 // leaves idle and the queue keeps them all busy until it is drained,
 // whatever the mix of sequence lengths.  Decode items that span several
 // partitions are combined afterwards by decode_reduce_kernel.
@@ -149,11 +153,23 @@ __device__ __forceinline__ void merge_item_two_pass(float* mg, float (&o)[Tiles:
   accumulate(2);                          // warps 2 and 3, then the output
 }
 
+// Work item i of the decode queue, in partition-major order: partition 0 of
+// every (sequence, KV head), then partition 1, and so on, so the last items
+// handed out are the late partitions of the longest sequences, most of them
+// shorter than a partition, and the workers finish close together.
+__device__ __forceinline__ void worker_item(const DecodeParams& p, int i, int& s, int& kvh,
+                                            int& part) {
+  const int per_part = p.num_seqs * p.num_kv_heads;
+  part = i / per_part;
+  const int r = i - part * per_part;
+  s = r / p.num_kv_heads;
+  kvh = r - s * p.num_kv_heads;
+}
+
 // A persistent decode worker (THREADS = 160 threads, `tid` 0..159): takes work
-// items i = atomicAdd(queue, 1) until i >= num_items; item i is partition
-// i % max_parts of KV head (i / max_parts) % Hkv of sequence
-// i / (max_parts * Hkv).  Items past a sequence's last partition are skipped
-// by the producer.  Every wait is bounded; a wait that gives up ends the
+// items i = atomicAdd(queue, 1) until i >= num_items (worker_item gives the
+// partition, KV head and sequence of i).  Items past a sequence's last
+// partition are skipped by the producer.  Every wait is bounded; a wait that gives up ends the
 // worker: the producer stops taking items and loading, the consumers stop at
 // the next item, and the producer drains its loads in flight before the
 // worker's threads leave (the error word says so).
@@ -175,7 +191,6 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
   volatile int* abort = cur_item + 1;
   float* mg = reinterpret_cast<float*>(smem + W::MERGE_OFF);
   const int warp = tid >> 5, lane = tid & 31;
-  const int per_seq = p.max_parts * p.num_kv_heads;
 
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -207,9 +222,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
         if (lane == 0) it = atomicAdd(queue, 1);
         it = __shfl_sync(0xffffffffu, it, 0);
         if (it >= num_items) break;
-        part = it % p.max_parts;
-        kvh = (it / p.max_parts) % p.num_kv_heads;
-        s = it / per_seq;
+        worker_item(p, it, s, kvh, part);
         const int L = decode_len<BS>(p, s, lane == 0 && part == 0 && kvh == 0);
         const int nblk_seq = (L + BS - 1) / BS;
         if (part < decode_parts(nblk_seq, p.part_blocks)) {
@@ -253,9 +266,8 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     named_barrier(bar_consumers, NW * 32);
     const int item = *cur_item;
     if (item < 0) break;
-    const int part = item % p.max_parts;
-    const int kvh = (item / p.max_parts) % p.num_kv_heads;
-    const int s = item / per_seq;
+    int s, kvh, part;
+    worker_item(p, item, s, kvh, part);
     const int L = decode_len<BS>(p, s, false);
     const int nblk_seq = (L + BS - 1) / BS;
     const int nparts = decode_parts(nblk_seq, p.part_blocks);
@@ -317,8 +329,16 @@ struct MixedShape {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
+// Launch order of the mixed grid (every count even: CTA pairs share a TPC):
+//   [0, lead)                          prefill slots 0 .. lead - 1
+//   [lead, lead + early)               decode CTAs started with the first tiles
+//   [lead + early, prefill_slots + early)  prefill slots lead ..
+//   [prefill_slots + early, grid)      decode CTAs that start as the tiles end
 struct MixedPlan {
-  int prefill_ctas;       // CTAs [0, prefill_ctas) run prefill tiles
+  int prefill_ctas;       // prefill tiles
+  int prefill_slots;      // prefill_ctas rounded up to even
+  int lead;               // prefill slots launched before the early decode CTAs
+  int early;              // decode CTAs launched with the first prefill tiles
   int prefill_tiles;      // 256-row tiles per prefill sequence (from max_q_len)
   int first_prefill_seq;  // == number of decode sequences
   int decode_items;       // num_decode * num_kv_heads * max_parts
@@ -335,13 +355,21 @@ __global__ void __launch_bounds__(MixedShape<T, BS, NT>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  // the split-KV combine that follows may be launched (it waits for this grid)
+  griddep_launch_dependents();
   const int b = blockIdx.x;
-  if (b < plan.prefill_ctas) {
-    // the last tile of a chunk sees the most keys: hand those out first
-    const int tile = plan.prefill_tiles - 1 - b % plan.prefill_tiles;
-    const int rest = b / plan.prefill_tiles;
-    const int h = rest % pp.num_q_heads;
-    const int s = plan.first_prefill_seq + rest / pp.num_q_heads;
+  const bool is_early = b >= plan.lead && b < plan.lead + plan.early;
+  // prefill slot of this CTA, or its index among the decode CTAs
+  const int slot = b < plan.lead ? b : b - plan.early;
+  if (!is_early && slot < plan.prefill_slots) {
+    if (slot >= plan.prefill_ctas) return;  // the spare slot of an odd count
+    // per chunk, the tile that sees the most keys first; query heads h and
+    // h + 1 of one tile side by side, so a CTA pair (one TPC) runs two
+    // tiles of the same length over the same K/V
+    const int h = slot % pp.num_q_heads;
+    const int rest = slot / pp.num_q_heads;
+    const int tile = plan.prefill_tiles - 1 - rest % plan.prefill_tiles;
+    const int s = plan.first_prefill_seq + rest / plan.prefill_tiles;
     prefill_tile<T, BS, Sh::SOFT_REGS, Sh::PROD_REGS>(&tm_q, &tm_k, &tm_v, pp, smem, tile, h, s);
     return;
   }
@@ -351,7 +379,8 @@ __global__ void __launch_bounds__(MixedShape<T, BS, NT>::THREADS, 1)
   // decode rows: sequence s must own exactly query row s
   if (w == 0 && tid == 0) {
     const int nd = plan.first_prefill_seq;
-    for (int s = b - plan.prefill_ctas; s < nd; s += gridDim.x - plan.prefill_ctas)
+    const int d = is_early ? b - plan.lead : b - plan.prefill_slots;  // decode CTA index
+    for (int s = d; s < nd; s += gridDim.x - plan.prefill_slots)
       if (pp.cu_q_lens[s] != s || pp.cu_q_lens[s + 1] != s + 1) record_error(PA_DEVERR_SEQ_RANGE);
   }
   decode_worker<typename Sh::Tiles, BS, NT>(&tm_k, &tm_v, dp, smem + w * Sh::Wk::BYTES,

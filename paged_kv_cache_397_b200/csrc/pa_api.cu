@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <type_traits>
 #include <climits>
@@ -374,6 +375,13 @@ size_t mixed_workspace_bytes(int num_decode, int num_q_heads, int head_dim, int 
 }
 
 
+// Share of the SMs the first prefill tiles of a mixed launch take (the rest
+// start decode workers).  Tuned on B200 for 256 decode rows over U[128, 4096]
+// cached tokens beside four 512-row chunks over 8192 cached tokens: prefill
+// there is ~58 % of the launch's SM time when decode runs at the SMs'
+// unsaturated rate.
+constexpr double kMixedPrefillShare = 7.0 / 12.0;
+
 template <typename T, int BS, int NT>
 pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const pa::PrefillParams& pp, const pa::DecodeParams& dp,
@@ -386,21 +394,38 @@ pa_status run_mixed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   if (pa_status st = configure_kernel(configured, kern, Sh::SMEM_BYTES, Sh::MIN_LAUNCH_REGS);
       st != PA_OK)
     return st;
-  // persistent decode workers: at most one CTA (two workers) per SM
+  // persistent decode workers: at most one CTA per SM; clusters of two CTAs
+  // (one TPC each), so every count is even
+  const int n_sm = sm_count() & ~1;
   long long decode_ctas = ((long long)plan.decode_items + Sh::WORKERS - 1) / Sh::WORKERS;
-  if (decode_ctas > sm_count()) decode_ctas = sm_count();
-  const long long grid = plan.prefill_ctas + decode_ctas;
+  if (decode_ctas > n_sm) decode_ctas = n_sm;
+  decode_ctas = (decode_ctas + 1) & ~1LL;
+  const long long grid = plan.prefill_slots + decode_ctas;
+  // The first prefill tiles take kMixedPrefillShare of the SMs and decode
+  // workers start on the rest at once, so the HBM-bound decode runs beside the
+  // tensor-bound tiles; later tiles follow on the SMs the first ones free, and
+  // the remaining decode CTAs start as the tiles run out (decode workers that
+  // find the queue empty exit, handing their SMs to the next tiles).
+  pa::MixedPlan pl = plan;
+  pl.lead = (int)std::min<long long>(plan.prefill_slots,
+                                     (long long)(n_sm * kMixedPrefillShare) & ~1LL);
+  pl.early = (int)std::min<long long>(decode_ctas, n_sm - pl.lead);
   if (grid <= 0) return PA_OK;
   if (grid > INT_MAX) return PA_ERR_INVALID_ARG;
-  kern<<<(unsigned)grid, Sh::THREADS, Sh::SMEM_BYTES, stream>>>(mq, mk, mv, pp, dp, plan);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (plan.decode_items > 0 && dp.max_parts > 1) {
-    const int units = dp.num_seqs * dp.num_q_heads;
-    pa::decode_reduce_kernel<T, 128>
-        <<<(units + pa::REDUCE_WARPS - 1) / pa::REDUCE_WARPS, pa::REDUCE_WARPS * 32, 0, stream>>>(
-            dp, BS);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(Sh::THREADS);
+  cfg.dynamicSmemBytes = Sh::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp, dp, pl) != cudaSuccess) return PA_ERR_CUDA;
+  if (plan.decode_items > 0 && dp.max_parts > 1) return launch_combine<T, 128>(dp, BS, stream);
   return PA_OK;
 }
 
@@ -996,7 +1021,7 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
   const long long tiles = (num_prefill > 0 && max_q_len > 0) ? (max_q_len + 255) / 256 : 0;
   const long long prefill_ctas = tiles * num_q_heads * num_prefill;
   const long long decode_items = (long long)num_decode * num_kv_heads * num_parts;
-  if (prefill_ctas > INT_MAX || decode_items > INT_MAX) return PA_ERR_INVALID_ARG;
+  if (prefill_ctas >= INT_MAX || decode_items > INT_MAX) return PA_ERR_INVALID_ARG;
 
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
@@ -1053,6 +1078,7 @@ pa_status pa_mixed_attention(void* out, const void* query, const void* key_cache
 
   pa::MixedPlan plan;
   plan.prefill_ctas = (int)prefill_ctas;
+  plan.prefill_slots = (int)((prefill_ctas + 1) & ~1LL);
   plan.prefill_tiles = (int)(tiles > 0 ? tiles : 1);
   plan.first_prefill_seq = num_decode;
   plan.decode_items = (int)decode_items;
