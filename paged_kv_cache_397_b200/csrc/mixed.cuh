@@ -9,28 +9,30 @@
 // decode row is the one-row case: it sees ctx_lens[s] + 1 tokens.
 //
 // How (B200 design).  The first num_decode sequences are decode rows (one
-// query each, at row s); the rest are prefill chunks.  One grid of 384-thread
-// CTAs covers both kinds of work:
-//  * CTAs [0, prefill_ctas) each run one 256-row prefill tile on the tcgen05
-//    tensor cores (prefill_tile, the same code as pa_prefill_chunk), longest
-//    tiles first;
-//  * the remaining CTAs (at most one per SM) each host two persistent decode
-//    workers of 160 threads (a producer warp and four consumer warps, on
-//    their own named barriers and shared memory).  A worker's producer takes
-//    split-KV work items (partition, KV head, decode sequence) from an atomic
-//    queue in the workspace and streams their (block, KV head) tiles through
-//    one TMA ring without draining it between items; the consumers process
-//    each item exactly as pa_decode's CTA does (same warp for each block, same
-//    merge order), so the results are bit-identical to pa_decode.
-// The grid runs as clusters of two CTAs, which share a TPC (the two SMs of a
-// tcgen05 CTA pair), and both CTAs of a cluster do the same kind of work: on
-// B200 a prefill tile whose TPC partner SM ran decode workers was measured
-// at about half speed, so a TPC runs two prefill tiles or two decode CTAs,
-// never one of each.  The hardware hands out clusters in launch order, so
-// the long compute-bound prefill tiles start first; decode workers start on the SMs the prefill tail
-// leaves idle and the queue keeps them all busy until it is drained,
-// whatever the mix of sequence lengths.  Decode items that span several
-// partitions are combined afterwards by decode_reduce_kernel.
+// query each, at row s); the rest are prefill chunks.  One grid of CTAs (512
+// threads with one query n-tile, 384 with two) covers both kinds of work:
+//  * a prefill CTA runs one 256-row prefill tile on the tcgen05 tensor cores
+//    (prefill_tile, the same code as pa_prefill_chunk);
+//  * a decode CTA (at most one per SM) hosts persistent decode workers of 160
+//    threads (a producer warp and four consumer warps, on their own named
+//    barriers and shared memory).  A worker's producer takes split-KV work
+//    items (partition, KV head, decode sequence) from an atomic queue in the
+//    workspace and streams their (block, KV head) tiles through one TMA ring
+//    without draining it between items; the consumers process each item
+//    exactly as pa_decode's CTA does (same warp for each block, same merge
+//    order), so the results are bit-identical to pa_decode.
+// Launch order (MixedPlan): a leading share of the prefill tiles, decode CTAs
+// for the other SMs, the remaining tiles, then the remaining decode CTAs.
+// The hardware hands out clusters in order, so the tensor-bound tiles and the
+// HBM-bound decode run side by side from the start; later tiles take the SMs
+// the first ones free, the last decode CTAs take the SMs the tiles leave, and
+// the queue keeps every worker busy until it is drained.  The grid runs as
+// clusters of two CTAs, which share a TPC (the two SMs of a tcgen05 CTA
+// pair), and both CTAs of a cluster do the same kind of work: on B200 a
+// prefill tile whose TPC partner SM ran decode workers was measured at about
+// half speed, so a TPC runs two prefill tiles or two decode CTAs, never one
+// of each.  Decode items that span several partitions are combined
+// afterwards by decode_reduce_kernel.
 #pragma once
 
 #include "decode.cuh"

@@ -5,7 +5,8 @@ Against the fp64 oracle (the chunk rule of "vLLM PagedAttention Deep Dive",
 chunk), bit-identical to running pa_decode and pa_prefill_chunk (without the
 key-range split of its last wave) separately on the two halves of the batch, bit-identical under relabelling of physical
 blocks, and at the full mixed workload (256 decode rows + 4 x 512-row chunks
-over 8192 cached tokens) on sampled rows."""
+over 8192 cached tokens) on sampled rows against the oracle and on every row
+against the two calls."""
 import numpy as np
 import pytest
 import torch
@@ -98,6 +99,23 @@ def test_mixed_is_bitwise_the_two_calls(decode_ctx, prefill_ctx, prefill_q):
         a = run_mixed(p, d, pt)
         b = run_separately(p, d, pt)
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("num_decode,prefill_ctx,prefill_q", [
+    (256, (8192,) * 4, (512,) * 4),   # the full mixed workload: every row compared
+    (6, (0, 900, 3000), (512, 300, 600)),  # more tiles than the leading share, few decode items
+    (300, (100,), (1,)),               # decode CTAs beyond the early share, one tile
+])
+def test_mixed_launch_order_is_bitwise_the_two_calls(num_decode, prefill_ctx, prefill_q):
+    # Grid order: a leading share of prefill tiles, decode CTAs started beside
+    # them, the remaining tiles, then the rest of the decode CTAs (all in CTA
+    # pairs).  Every row must still equal the separate calls bit for bit.
+    p = synth.mixed_batch(seed=71, num_decode=num_decode, prefill_ctx=list(prefill_ctx),
+                          prefill_q=list(prefill_q))
+    d = gpu_inputs(p)
+    a = run_mixed(p, d, 1024)
+    b = run_separately(p, d, 1024)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
 def test_mixed_bit_identical_under_block_relabelling():
