@@ -55,8 +55,9 @@ struct WorkerShape {
   static constexpr int BAR_OFF = MERGE_OFF + MERGE_BYTES;
   static constexpr int NBAR = 2 * Dc::NS + 2 * QD;
   static constexpr int ITEM_OFF = BAR_OFF + NBAR * 8;
-  // item slots, the current item, the worker's abort word
-  static constexpr int BYTES = (ITEM_OFF + (QD + 2) * 4 + 1023) / 1024 * 1024;
+  // item slots, the current item, the worker's abort word, the last ring
+  // position filled on each stage
+  static constexpr int BYTES = (ITEM_OFF + (QD + 2 + Dc::NS) * 4 + 1023) / 1024 * 1024;
 };
 
 // Merge of one item's four consumer-warp states for a decode worker, through
@@ -171,7 +172,16 @@ __device__ __forceinline__ void worker_item(const DecodeParams& p, int i, int& s
 // A persistent decode worker (THREADS = 160 threads, `tid` 0..159): takes work
 // items i = atomicAdd(queue, 1) until i >= num_items (worker_item gives the
 // partition, KV head and sequence of i).  Items past a sequence's last
-// partition are skipped by the producer.  Every wait is bounded; a wait that gives up ends the
+// partition are skipped by the producer.  The ring runs on across items: the
+// producer fills each item's first NS positions, and after that every
+// consumer warp refills the stage it has just read with its own next
+// position of the item (position i + NS of an item is read by the warp that
+// read position i), so no warp waits behind a slower one's stage.  Every
+// position read is released on its stage's empty barrier, in position order
+// per stage; before the producer fills position q it waits until position
+// q - NS has been filled (last_fill, written after the release of q - 2NS)
+// and then for that position's release, so its parity wait cannot alias a
+// phase two back.  Every wait is bounded; a wait that gives up ends the
 // worker: the producer stops taking items and loading, the consumers stop at
 // the next item, and the producer drains its loads in flight before the
 // worker's threads leave (the error word says so).
@@ -183,7 +193,8 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
   using Shape = DecodeShape<Tiles, BS, NT>;
   using W = WorkerShape<Tiles, BS, NT>;
   using T = typename Tiles::Elem;
-  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS, QD = W::QD;
+  constexpr int D = Shape::D, NW = Shape::NW, NS = Shape::NS, QD = W::QD, SB = Shape::SB;
+  static_assert(NS % NW == 0 && NS * SB <= 32, "refills stay on one warp; one table load per lane");
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + W::BAR_OFF);
   uint64_t* empty_bar = full_bar + NS;
   uint64_t* item_full = empty_bar + NS;
@@ -191,6 +202,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + W::ITEM_OFF);
   volatile int* cur_item = item_slot + QD;
   volatile int* abort = cur_item + 1;
+  volatile int* last_fill = abort + 1;  // [NS]: last ring position filled per stage
   float* mg = reinterpret_cast<float*>(smem + W::MERGE_OFF);
   const int warp = tid >> 5, lane = tid & 31;
 
@@ -203,6 +215,7 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], 1);
     }
+    for (int i = 0; i < NS; ++i) last_fill[i] = -1;
     *abort = 0;
     fence_barrier_init();
   }
@@ -241,18 +254,64 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
       }
       alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
       if (item < 0 || !alive) break;
-      const int next = produce_item<Tiles, BS, NT>(
-          tm_k, tm_v, p, smem, full_bar, empty_bar,
-          p.block_tables + (size_t)s * p.max_blocks_per_seq, kvh, part * p.part_blocks, nblk, g,
-          lane, policy, alive, abort);
-      g = __shfl_sync(0xffffffffu, next, 0);  // lane 0's count (the lanes agree unless aborted)
+      // the item's first NS positions (its consumers refill the rest)
+      const int nstages = (nblk + SB - 1) / SB;
+      const int nhead = min(nstages, NS);
+      const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + part * p.part_blocks;
+      int phys = 0;
+      if (lane < nhead * SB && lane < nblk) {
+        phys = __ldg(bt + lane);
+        if (phys < 0 || phys >= p.num_blocks) {
+          record_error(PA_DEVERR_BLOCK_RANGE);
+          phys = 0;
+        }
+      }
+      for (int i = 0; i < nhead; ++i) {
+        int ph[SB];
+#pragma unroll
+        for (int u = 0; u < SB; ++u) ph[u] = __shfl_sync(0xffffffffu, phys, (i * SB + u) & 31);
+        if (lane == 0 && alive) {
+          const int q = g + i, st = q % NS;
+          if (q >= NS) {
+            // position q - NS filled (so q - 2NS released), then q - NS released
+            const uint64_t t0 = global_timer_ns();
+            while (last_fill[st] < q - NS && alive) {
+              if (*abort) alive = false;
+              else if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                record_error(PA_DEVERR_WAIT_TIMEOUT);
+                alive = false;
+              }
+            }
+            if (alive) alive = mbar_wait(&empty_bar[st], ((q / NS) - 1) & 1, abort);
+          }
+          if (alive) {
+            const int nb = min(SB, nblk - i * SB);
+            mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
+            uint8_t* sk = smem + st * Shape::STAGE_BYTES;
+#pragma unroll
+            for (int u = 0; u < SB; ++u)
+              if (u < nb)
+                Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
+                             (ph[u] * p.num_kv_heads + kvh) * BS, u, &full_bar[st], policy);
+            last_fill[st] = q;
+          }
+        }
+      }
+      alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
+      g += nstages;
     }
     named_barrier(bar_all, Shape::THREADS);  // the consumers are done
-    if (*abort && lane == 0) drain_ring<NS>(full_bar, g);
+    if (*abort && lane == 0) {
+      // let every load still in flight land before the worker's threads leave
+      for (int st = 0; st < NS; ++st)
+        if (last_fill[st] >= 0) mbar_drain(&full_bar[st], (last_fill[st] / NS) & 1);
+    }
     return;
   }
 
   // -------------------------------------------------------------- consumers
+  const uint64_t policy = l2_policy_evict_first();
   // One thread takes each item from its slot and hands it to all four warps
   // through cur_item, so the warps always agree on the item (and so reach
   // the same named barriers) even if a wait times out.
@@ -288,13 +347,57 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
     // a stage may reach past the item's last block (into the next partition)
     const int L_end = min(L, (blk0 + nblk) * BS);
     bool alive = true;
+    const int32_t* bt = p.block_tables + (size_t)s * p.max_blocks_per_seq + blk0;
+    int ids[SB];  // lane l: the blocks of this warp's (kw + l)-th position of the item
+    int kw = -32;
     for (int i = warp; i < nstages; i += NW) {
       const int gi = g + i, st = gi % NS;
+      // after a wait gave up the warp still runs through its (garbage) stages,
+      // every lane alike, so the .aligned loads and MMAs stay converged
       if (alive) alive = mbar_wait(&full_bar[st], (gi / NS) & 1, abort);
       consume_block<Tiles, BS, NT>(o, m_run, l_run, qf, smem + st * Shape::STAGE_BYTES,
-                                   (blk0 + i * Shape::SB) * BS, L_end, p.scale_log2, lane);
+                                   (blk0 + i * SB) * BS, L_end, p.scale_log2, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
+      const int nxt = i + NS;  // this warp's next position on stage st (warp-uniform test)
+      if (nxt < nstages) {
+        const int kk = (nxt - warp) / NW;
+        if (kk >= kw + 32) {
+          kw = kk;
+#pragma unroll
+          for (int u = 0; u < SB; ++u) {
+            const int b = (warp + NW * (kk + lane)) * SB + u;
+            int id = 0;
+            if (b < nblk) {
+              id = __ldg(bt + b);
+              if (id < 0 || id >= p.num_blocks) {
+                record_error(PA_DEVERR_BLOCK_RANGE);
+                id = 0;
+              }
+            }
+            ids[u] = id;
+          }
+        }
+        int ph[SB];
+#pragma unroll
+        for (int u = 0; u < SB; ++u) ph[u] = __shfl_sync(0xffffffffu, ids[u], kk - kw);
+        if (lane == 0 && alive) {
+          // the warp's reads of the stage are done (__syncwarp above); order
+          // them before the async-proxy writes that refill it
+          fence_proxy_async_smem();
+          const int nb = min(SB, nblk - nxt * SB);
+          mbar_arrive_expect_tx(&full_bar[st], nb * Shape::BLOCK_BYTES);
+          uint8_t* sk = smem + st * Shape::STAGE_BYTES;
+#pragma unroll
+          for (int u = 0; u < SB; ++u)
+            if (u < nb)
+              Tiles::issue(sk, sk + Shape::TILE_BYTES, tm_k, tm_v,
+                           (ph[u] * p.num_kv_heads + kvh) * BS, u, &full_bar[st], policy);
+          // the release of gi above is visible before this position is
+          __threadfence_block();
+          last_fill[st] = g + nxt;
+        }
+      }
     }
     g += nstages;
     // the opening barrier of merge_item also orders this item's read of
