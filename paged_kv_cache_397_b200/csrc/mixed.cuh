@@ -411,9 +411,9 @@ __device__ __forceinline__ void decode_worker(const CUtensorMap* tm_k, const CUt
 // CTA shape of the mixed launch.  With one query n-tile (groups up to 8) a
 // CTA of 16 warps hosts three decode workers, 12 consumer warps per SM as
 // three pa_decode CTAs have, and a prefill tile's softmax warpgroups get 200
-// registers by taking the other two warpgroups down to 56 (2 x 128 x 200 +
-// 256 x 56 = 512 x 128).  With two n-tiles the consumers need more registers:
-// 12 warps and two workers.
+// registers, its producer warpgroup 88 and the idle fourth warpgroup 24
+// (2 x 128 x 200 + 128 x 88 + 128 x 24 = 512 x 128).  With two n-tiles the
+// consumers need more registers: 12 warps and two workers.
 template <typename T, int BS, int NT>
 struct MixedShape {
   using Pf = PrefillShape<T, BS>;
@@ -423,9 +423,11 @@ struct MixedShape {
   static constexpr int THREADS = NT == 1 ? 512 : Pf::THREADS;
   static constexpr int WORKERS = THREADS / Dc::THREADS;  // decode workers per CTA
   static constexpr uint32_t SOFT_REGS = Pf::SOFTMAX_REGS;
-  static constexpr uint32_t PROD_REGS = NT == 1 ? 56 : Pf::PRODUCER_REGS;
+  static constexpr uint32_t PROD_REGS = NT == 1 ? 88 : Pf::PRODUCER_REGS;
+  static constexpr uint32_t IDLE_REGS = NT == 1 ? 24 : PROD_REGS;  // warps 12-15
   static constexpr int MIN_LAUNCH_REGS = NT == 1 ? 128 : Pf::MIN_LAUNCH_REGS;
-  static_assert(2 * 128 * SOFT_REGS + (THREADS - 256) * PROD_REGS <= THREADS * MIN_LAUNCH_REGS,
+  static_assert(2 * 128 * SOFT_REGS + 128 * PROD_REGS + (THREADS - 384) * IDLE_REGS <=
+                    THREADS * MIN_LAUNCH_REGS,
                 "register split exceeds the launch allocation");
   static constexpr int DEC_SMEM = 1024 + WORKERS * Wk::BYTES;
   static constexpr int SMEM_BYTES = Pf::SMEM_BYTES > DEC_SMEM ? Pf::SMEM_BYTES : DEC_SMEM;
@@ -475,7 +477,8 @@ __global__ void __launch_bounds__(MixedShape<T, BS, NT>::THREADS, 1)
     const int rest = slot / pp.num_q_heads;
     const int tile = plan.prefill_tiles - 1 - rest % plan.prefill_tiles;
     const int s = plan.first_prefill_seq + rest / plan.prefill_tiles;
-    prefill_tile<T, BS, Sh::SOFT_REGS, Sh::PROD_REGS>(&tm_q, &tm_k, &tm_v, pp, smem, tile, h, s);
+    prefill_tile<T, BS, Sh::SOFT_REGS, Sh::PROD_REGS, 128, Sh::IDLE_REGS>(&tm_q, &tm_k, &tm_v, pp,
+                                                                          smem, tile, h, s);
     return;
   }
   const int w = threadIdx.x / Sh::Dc::THREADS;

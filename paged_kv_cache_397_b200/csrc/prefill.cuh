@@ -219,10 +219,12 @@ __device__ __forceinline__ void prefill_p_chunks(const uint32_t (&sv)[128], uint
 // `slot`; the parts' partial rows are combined by the last one to finish).
 // Needs every thread of the CTA (12 warps, or more: warps past the producer
 // warpgroup idle), 1024-byte aligned shared memory at `smem` and all 512
-// tensor-memory columns.  SOFT_REGS / PROD_REGS: the setmaxnreg split between
-// the two softmax warpgroups and every other warpgroup of the CTA.
+// tensor-memory columns.  SOFT_REGS / PROD_REGS / IDLE_REGS: the setmaxnreg
+// split between the two softmax warpgroups, the producer warpgroup and any
+// warpgroup past it.
 template <typename T, int BS, uint32_t SOFT_REGS = PrefillShape<T, BS>::SOFTMAX_REGS,
-          uint32_t PROD_REGS = PrefillShape<T, BS>::PRODUCER_REGS, int HEAD_DIM = 128>
+          uint32_t PROD_REGS = PrefillShape<T, BS>::PRODUCER_REGS, int HEAD_DIM = 128,
+          uint32_t IDLE_REGS = PROD_REGS>
 __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                              const CUtensorMap* tm_v, const PrefillParams& p,
                                              uint8_t* smem, int tile, int h, int s, int part = 0,
@@ -304,7 +306,10 @@ __device__ __forceinline__ void prefill_tile(const CUtensorMap* tm_q, const CUte
   const uint32_t tmem = *tmem_slot;
 
   int armed = 0;  // TMA warp: ring items (K_j = 2j, V_j = 2j + 1) armed so far
-  if (warp >= 8) {
+  if (warp >= 12) {
+    // warpgroups past the producer warpgroup (a CTA of the mixed launch): idle
+    setmaxnreg_dec<IDLE_REGS>();
+  } else if (warp >= 8) {
     // producer warpgroup: TMA warp, MMA warp, two idle warps
     setmaxnreg_dec<PROD_REGS>();
   if (warp == Sh::TMA_WARP) {
