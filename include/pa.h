@@ -462,8 +462,8 @@ pa_status pa_prefill_chunk(void *out, const void *query, const void *key_cache,
  *                 partials.  Calls sharing a workspace must be ordered.
  * One kernel launch covers both kinds of rows (plus the split-KV combine of
  * the decode rows when they span several partitions, and the 4-byte memset
- * of the queue counter).  head_dim must be 128; fp16 / bf16 caches;
- * group <= 16.
+ * of the queue counter); it runs as clusters of two CTAs, one TPC each.
+ * head_dim must be 128; fp16 / bf16 caches; group <= 16.
  */
 pa_status pa_mixed_workspace_size(int num_decode_seqs, int num_q_heads, int num_kv_heads,
                                   int head_dim, int block_size, int max_ctx_len,
