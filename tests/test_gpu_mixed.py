@@ -118,6 +118,20 @@ def test_mixed_launch_order_is_bitwise_the_two_calls(num_decode, prefill_ctx, pr
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_mixed_odd_tile_count():
+    # 5 query heads over one KV head: an odd number of prefill tiles, so the
+    # last CTA pair holds one tile and one spare slot
+    p = small_batch(83, 16, torch.bfloat16, 5, 1, decode_ctx=(7, 300, 2500), prefill_ctx=(40,),
+                    prefill_q=(200,))
+    d = gpu_inputs(p)
+    a = run_mixed(p, d, 256)
+    b = run_separately(p, d, 256)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    oracle_scatter_chunks(p)
+    ref, _ = chunk_reference(p)
+    assert max_err(a.cpu(), ref) <= TOL[p.dtype]
+
+
 def test_mixed_bit_identical_under_block_relabelling():
     p = small_batch(52, 16, torch.bfloat16, 8, 2)
     out_a = run_mixed(p, gpu_inputs(p)).cpu()
